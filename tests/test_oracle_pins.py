@@ -1,0 +1,375 @@
+"""Pins of the CPU oracle to facts fixed outside it.
+
+Each test ties one oracle function to something it does not compute itself:
+hand-worked examples (tests/golden/hand_examples.json), closed forms that
+reduce to a library routine (numpy matmul / mean, torch's fp32->bf16
+rounding), invariants of the definitions, and brute force over all subsets on
+tiny rows.  The cases are chosen so that a dropped term, a wrong sign or
+index, a transposed operand or an off-by-one in the causal limit fails one.
+"""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from workloads import Batch
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")))
+
+
+def make_batch(Q, K, W, q_lens, k_lens, pos, **params):
+    Q = torch.as_tensor(np.asarray(Q, np.float32)).to(torch.bfloat16)
+    K = torch.as_tensor(np.asarray(K, np.float32)).to(torch.bfloat16)
+    W = torch.as_tensor(np.asarray(W, np.float32))
+    off = lambda ls: torch.tensor(np.concatenate([[0], np.cumsum(ls)]), dtype=torch.int32)
+    return Batch(Q, K, W, off(q_lens), off(k_lens), torch.tensor(pos, dtype=torch.int32), dict(params))
+
+
+def ref_topk(scores, k):
+    """Order by score desc, index asc (np.lexsort: last key is primary)."""
+    n = len(scores)
+    order = np.lexsort((np.arange(n), -np.asarray(scores)))
+    out = list(order[:k]) + [-1] * max(0, k - n)
+    return out
+
+
+# ------------------------------------------------------------ hand examples
+
+def test_dense_hand_example():
+    g = GOLD["dense"]
+    qs = g["queries"]
+    b = make_batch([q["q"] for q in qs], g["K"], [q["w"] for q in qs], [len(qs)], [len(g["K"])],
+                   [q["pos"] for q in qs])
+    for r, q in enumerate(qs):
+        res = oracle.dense(b, rows=[r], k=len(q["scores"]), want_all=True)
+        n = len(q["scores"])
+        assert res["all"][0][:n].tolist() == q["scores"]
+        assert np.all(np.isneginf(res["all"][0][n:]))
+        for k, expect in q["topk"].items():
+            out = oracle.dense(b, rows=[r], k=int(k))["idx"][0].tolist()
+            assert out == expect, (r, k, out, expect)
+
+
+def test_pivot_hand_example():
+    g = GOLD["pivot"]
+    qs = g["group"]
+    b = make_batch([q["q"] for q in qs], g["K"], [q["w"] for q in qs], [len(qs)], [len(g["K"])],
+                   [q["pos"] for q in qs])
+    for case in g["cases"]:
+        res = oracle.pivot(b, G=2, C=case["C"], k=case["k"])
+        assert res["proxy_q"][0].tolist() == g["proxy_q"]
+        assert res["proxy_w"][0].tolist() == g["proxy_w"]
+        n = len(case["cand"])
+        assert res["cand"][0][:n].tolist() == case["cand"]
+        assert res["cand_score"][0][:n].tolist() == [g["proxy_scores"][s] for s in case["cand"]]
+        for j in range(2):
+            assert res["reuse_idx"][j].tolist() == case["reuse"][j], case
+            assert sorted(res["refine_idx"][j].tolist()) == sorted(case["refine"][j]), case
+
+
+def test_hisa_hand_example():
+    g = GOLD["hisa"]
+    q = g["query"]
+    b = make_batch([q["q"]], g["K"], [q["w"]], [1], [len(g["K"])], [q["pos"]])
+    pooled = oracle.hisa_pool(b, g["block"])
+    assert pooled.tolist() == g["pooled"]
+    for case in g["cases"]:
+        res = oracle.hisa(b, g["block"], case["keep"], case["k"])
+        kept = [x for x in res["kept"][0].tolist() if x >= 0]
+        assert kept == case["kept"], case
+        assert sorted(res["idx"][0].tolist()) == sorted(case["topk"]), case
+
+
+# ------------------------------------------------- closed forms / library
+
+def test_nonnegative_dots_reduce_to_matmul():
+    """If every q.k >= 0 the ReLU is inactive: I[t,s] = (sum_h w[t,h] q[t,h]) . k[s]."""
+    g = torch.Generator().manual_seed(7)
+    T, H, d = 40, 5, 12
+    Q = torch.randint(0, 4, (T, H, d), generator=g).float().numpy()
+    K = torch.randint(0, 4, (T, d), generator=g).float().numpy()
+    W = (torch.randint(-4, 5, (T, H), generator=g).float() / 4).numpy()
+    b = make_batch(Q, K, W, [T], [T], list(range(T)))
+    got = oracle.dense(b, k=T, want_all=True)["all"]
+    expect = np.einsum("th,thd->td", W.astype(np.float64), Q.astype(np.float64)) @ K.astype(np.float64).T
+    mask = np.tril(np.ones((T, T), bool))
+    assert np.array_equal(got[mask], expect[mask])
+    assert np.all(np.isneginf(got[~mask]))
+
+
+def test_nonpositive_dots_give_zero_and_index_order():
+    """q >= 0, k <= 0: every ReLU is 0, all scores tie at 0, top-k is the k lowest indices."""
+    T, H, d, k = 30, 3, 8, 7
+    Q = np.ones((T, H, d)); K = -(np.arange(T * d).reshape(T, d) % 5)
+    W = np.linspace(-1, 1, T * H).reshape(T, H)
+    b = make_batch(Q, K, W, [T], [T], list(range(T)))
+    res = oracle.dense(b, k=k, want_all=True)
+    mask = np.tril(np.ones((T, T), bool))
+    assert np.all(res["all"][mask] == 0)
+    for t in range(T):
+        n = min(k, t + 1)
+        assert res["idx"][t].tolist() == list(range(n)) + [-1] * (k - n)
+
+
+def test_monotone_keys_select_the_last_k():
+    """k[s] = s * 1, q = 1, w = 1: I = H*d*s grows with s, so the top-k is the last k eligible keys."""
+    T, H, d, k = 50, 2, 4, 6
+    Q = np.ones((T, H, d)); K = np.repeat(np.arange(T)[:, None], d, 1); W = np.ones((T, H))
+    b = make_batch(Q, K, W, [T], [T], list(range(T)))
+    res = oracle.dense(b, k=k, want_all=True)
+    for t in range(T):
+        assert res["all"][t][: t + 1].tolist() == [H * d * s for s in range(t + 1)]
+        n = min(k, t + 1)
+        assert res["idx"][t].tolist() == list(range(t, t - n, -1)) + [-1] * (k - n)
+
+
+def test_single_head_scalar_is_relu_product():
+    """H = 1, d = 1, w = 1: I = max(0, q*k)."""
+    rng = np.random.default_rng(3)
+    T = 25
+    q = rng.integers(-5, 6, T).astype(np.float64); kk = rng.integers(-5, 6, T).astype(np.float64)
+    b = make_batch(q.reshape(T, 1, 1), kk.reshape(T, 1), np.ones((T, 1)), [T], [T], list(range(T)))
+    got = oracle.dense(b, k=T, want_all=True)["all"]
+    for t in range(T):
+        assert got[t][: t + 1].tolist() == np.maximum(q[t] * kk[: t + 1], 0).tolist()
+
+
+def test_weight_sign_is_applied_after_relu():
+    """One head with w = -1: I = -max(0, q.k), never positive (a ReLU applied after w would differ)."""
+    T, d = 20, 4
+    rng = np.random.default_rng(5)
+    Q = rng.integers(-3, 4, (T, 1, d)); K = rng.integers(-3, 4, (T, d))
+    b = make_batch(Q, K, -np.ones((T, 1)), [T], [T], list(range(T)))
+    got = oracle.dense(b, k=T, want_all=True)["all"]
+    dots = Q[:, 0, :].astype(np.float64) @ K.T.astype(np.float64)
+    mask = np.tril(np.ones((T, T), bool))
+    assert np.array_equal(got[mask], (-np.maximum(dots, 0))[mask])
+
+
+def test_round_bf16_matches_torch_on_fp32_values():
+    """For fp32-representable inputs, torch's fp32 -> bf16 conversion (RNE, one rounding) is the reference."""
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(4000, generator=g) * torch.exp2(torch.randint(-30, 30, (4000,), generator=g).float())
+    # exact ties: 8 significant bits + a half-ulp bit
+    ties = (torch.randint(128, 256, (500,), generator=g).float() + 0.5) * torch.exp2(
+        torch.randint(-20, 20, (500,), generator=g).float())
+    x = torch.cat([x, ties, -ties])
+    expect = x.to(torch.bfloat16).to(torch.float64).numpy()
+    got = np.array([oracle.round_bf16(float(v)) for v in x.numpy()])
+    assert np.array_equal(got, expect)
+
+
+def test_round_bf16_rounds_doubles_directly():
+    """A double just above a bf16 tie rounds up; rounding through fp32 first would land on the tie and go to even."""
+    x = 1.0 + 2.0 ** -8 + 2.0 ** -40
+    assert oracle.round_bf16(x) == 1.0 + 2.0 ** -7
+    assert oracle.round_bf16(-x) == -(1.0 + 2.0 ** -7)
+    assert float(torch.tensor(x, dtype=torch.float64).to(torch.float32).to(torch.bfloat16)) == 1.0
+
+
+# ------------------------------------------------------------- invariants
+
+@pytest.fixture(scope="module")
+def tiny():
+    return workloads.tiny_integer(seed=0, T=96, H=4, d=32, k=20)
+
+
+def test_positive_weight_scaling(tiny):
+    r1 = oracle.dense(tiny, want_all=True)
+    b2 = Batch(tiny.Q, tiny.K, tiny.W * 4, tiny.q_offsets, tiny.k_offsets, tiny.q_pos, tiny.params)
+    r2 = oracle.dense(b2, want_all=True)
+    fin = np.isfinite(r1["all"])
+    assert np.array_equal(r2["all"][fin], 4 * r1["all"][fin])
+    assert np.array_equal(r1["idx"], r2["idx"])
+
+
+def test_head_permutation_and_zero_heads(tiny):
+    r1 = oracle.dense(tiny, want_all=True)
+    perm = torch.tensor([2, 0, 3, 1])
+    Q = torch.cat([tiny.Q[:, perm], tiny.Q[:, :1]], 1)          # extra head with weight 0
+    W = torch.cat([tiny.W[:, perm], torch.zeros(tiny.n_q, 1)], 1)
+    r2 = oracle.dense(Batch(Q, tiny.K, W, tiny.q_offsets, tiny.k_offsets, tiny.q_pos, tiny.params), want_all=True)
+    assert np.array_equal(r1["all"], r2["all"])
+
+
+def test_causality(tiny):
+    """Changing keys after a query's position leaves that query's row unchanged."""
+    t = 40
+    K2 = tiny.K.clone()
+    K2[t + 1:] = -K2[t + 1:] + 1
+    b2 = Batch(tiny.Q, K2, tiny.W, tiny.q_offsets, tiny.k_offsets, tiny.q_pos, tiny.params)
+    r1 = oracle.dense(tiny, rows=[t], want_all=True)
+    r2 = oracle.dense(b2, rows=[t], want_all=True)
+    assert np.array_equal(r1["all"], r2["all"]) and np.array_equal(r1["idx"], r2["idx"])
+    r3 = oracle.dense(b2, rows=[t + 1], want_all=True)
+    assert not np.array_equal(oracle.dense(tiny, rows=[t + 1], want_all=True)["all"], r3["all"])
+
+
+def test_position_clamp_and_empty_rows():
+    b = workloads.ragged(1, [3, 2], [5, 4], H=2, d=8, k=6, integer=True)
+    b.q_pos = torch.tensor([-1, 0, 9, 3, 100], dtype=torch.int32)
+    res = oracle.dense(b, want_all=True)
+    assert res["n_elig"].tolist() == [0, 1, 5, 4, 4]
+    assert res["idx"][0].tolist() == [-1] * 6
+    assert res["idx"][1].tolist() == [0] + [-1] * 5
+
+
+def test_selection_is_the_brute_force_best_subset():
+    """Top-k equals the best k-subset under (score desc, index asc), found by enumerating every subset."""
+    b = workloads.tiny_integer(seed=3, T=9, H=2, d=4, k=4)   # integer inputs: many ties
+    res = oracle.dense(b, k=4, want_all=True)
+    for t in range(b.n_q):
+        n = t + 1
+        sc = res["all"][t][:n]
+        kk = min(4, n)
+
+        def key(sub):   # larger is better: descending (score, -index) sequence
+            return sorted(((sc[i], -i) for i in sub), reverse=True)
+        best = max(itertools.combinations(range(n), kk), key=key)
+        assert sorted(res["idx"][t][:kk].tolist()) == sorted(best)
+        # ranking order inside the output
+        assert res["idx"][t][:kk].tolist() == ref_topk(sc, kk)[:kk]
+
+
+# ------------------------------------------------------------------ PIVOT
+
+def test_pivot_group_of_one_is_dense():
+    b = workloads.tiny_integer(seed=1, T=128, H=4, d=32, k=24)
+    d = oracle.dense(b, k=24)
+    p = oracle.pivot(b, G=1, C=24, k=24)
+    assert np.array_equal(p["reuse_idx"], d["idx"])
+    for t in range(b.n_q):
+        assert sorted(p["refine_idx"][t].tolist()) == sorted(d["idx"][t].tolist())
+
+
+def test_pivot_refine_with_full_candidates_is_dense():
+    b = workloads.ragged(2, [64, 37], [64, 50], H=4, d=16, k=10)
+    d = oracle.dense(b, k=10)
+    G = 8
+    p = oracle.pivot(b, G=G, C=64, k=10)
+    sizes = [8] * 8 + [8, 8, 8, 8, 5]            # seq 0: 64 = 8 groups; seq 1: 37 = 4 full + 5
+    assert p["refine_idx"].shape[0] == G * len(sizes)
+    t = 0
+    for g, size in enumerate(sizes):
+        for j in range(G):
+            if j < size:
+                assert np.array_equal(p["refine_idx"][g * G + j], d["idx"][t]), t
+                t += 1
+            else:
+                assert np.all(p["refine_idx"][g * G + j] == -1)
+    assert t == b.n_q
+
+
+def test_pivot_reuse_independent_of_candidate_count():
+    """Once C >= k + G - 1, Reuse equals the proxy top-k over each query's own prefix."""
+    b = workloads.tiny_integer(seed=4, T=200, H=4, d=32, k=12, signed_w=True)
+    G, k = 8, 12
+    small = oracle.pivot(b, G=G, C=k + G - 1, k=k)
+    full = oracle.pivot(b, G=G, C=200, k=k)
+    assert np.array_equal(small["reuse_idx"], full["reuse_idx"])
+
+
+def test_pivot_reuse_is_proxy_topk_over_own_prefix():
+    """Reuse for query t = the proxy's dense top-k over t's own prefix (C >= k + G - 1), so it is causal."""
+    b = workloads.tiny_integer(seed=8, T=96, H=4, d=32, k=10)
+    G, k = 8, 10
+    p = oracle.pivot(b, G=G, C=k + G - 1, k=k)
+    for g in range(96 // G):
+        pq = torch.as_tensor(p["proxy_q"][g], dtype=torch.float32).to(torch.bfloat16)
+        pw = torch.as_tensor(p["proxy_w"][g], dtype=torch.float32)
+        pos = b.q_pos[g * G:(g + 1) * G]
+        one = Batch(pq[None].expand(G, -1, -1).contiguous(), b.K, pw[None].expand(G, -1).contiguous(),
+                    torch.tensor([0, G], dtype=torch.int32), b.k_offsets, pos.clone())
+        d = oracle.dense(one, k=k)
+        assert np.array_equal(p["reuse_idx"][g * G:(g + 1) * G], d["idx"]), g
+        for j in range(G):
+            r = p["reuse_idx"][g * G + j]
+            assert np.all(r[r >= 0] <= int(pos[j]))
+
+
+def test_pivot_proxy_is_the_rounded_mean():
+    b = workloads.dense_prefill(seed=9, T=64, H=4, d=16, k=8)
+    G = 16
+    p = oracle.pivot(b, G=G, C=8, k=8)
+    Qd = b.Q.to(torch.float64).view(-1, G, 4, 16).mean(1)        # library mean in double
+    Wd = b.W.to(torch.float64).view(-1, G, 4).mean(1)
+    rounded = np.vectorize(oracle.round_bf16)(Qd.numpy())
+    assert np.array_equal(p["proxy_q"], rounded)
+    np.testing.assert_allclose(p["proxy_w"], Wd.numpy(), rtol=1e-15, atol=0)
+    # the rounded proxy differs from the unrounded mean somewhere, so rounding is really applied
+    assert not np.array_equal(rounded, Qd.numpy())
+
+
+def test_pivot_candidates_are_proxy_topc():
+    """The candidate set is the proxy's top-C over the group's scan range (proxy scored as a dense query)."""
+    b = workloads.tiny_integer(seed=5, T=64, H=2, d=8, k=5)
+    G, C = 4, 9
+    p = oracle.pivot(b, G=G, C=C, k=5)
+    for g in range(64 // G):
+        # group proxy as an explicit single-query batch over the same keys
+        pq = torch.as_tensor(p["proxy_q"][g], dtype=torch.float32).to(torch.bfloat16)[None]
+        pw = torch.as_tensor(p["proxy_w"][g], dtype=torch.float32)[None]
+        pos = int(b.q_pos[g * G + G - 1])
+        one = Batch(pq, b.K, pw, torch.tensor([0, 1], dtype=torch.int32), b.k_offsets,
+                    torch.tensor([pos], dtype=torch.int32))
+        d = oracle.dense(one, k=C)
+        assert sorted(x for x in d["idx"][0].tolist() if x >= 0) == \
+            [x for x in p["cand"][g].tolist() if x >= 0]
+
+
+def test_pivot_external_candidates_match_own():
+    b = workloads.tiny_integer(seed=6, T=96, H=4, d=32, k=10)
+    own = oracle.pivot(b, G=4, C=30, k=10)
+    ext = oracle.pivot(b, G=4, C=30, k=10, ext_cand=own["cand"])
+    for key in ("cand", "reuse_idx", "refine_idx"):
+        assert np.array_equal(own[key], ext[key])
+
+
+# ------------------------------------------------------------------- HISA
+
+def test_hisa_pool_is_block_mean():
+    b = workloads.ragged(3, [1, 1], [300, 77], H=2, d=8, k=4)
+    pooled = oracle.hisa_pool(b, 32)
+    K = b.K.to(torch.float64)
+    blocks = []
+    for s0, L in ((0, 300), (300, 77)):
+        for j in range(0, L, 32):
+            blocks.append(K[s0 + j: s0 + min(j + 32, L)].mean(0).numpy())
+    np.testing.assert_allclose(pooled, np.stack(blocks), rtol=1e-14, atol=1e-15)
+
+
+def test_hisa_keep_all_blocks_is_dense():
+    b = workloads.ragged(4, [3, 2], [500, 260], H=4, d=16, k=40, pos_mode="random")
+    d = oracle.dense(b, k=40)
+    h = oracle.hisa(b, B=16, keep=40, k=40)
+    for t in range(b.n_q):
+        assert sorted(h["idx"][t].tolist()) == sorted(d["idx"][t].tolist()), t
+
+
+def test_hisa_block_size_one_scores_tokens():
+    """B = 1: each pooled key is the key itself, so the block scores are the token scores."""
+    b = workloads.ragged(5, [2], [40], H=3, d=8, k=5)
+    h = oracle.hisa(b, B=1, keep=3, k=5)
+    d = oracle.dense(b, k=5, want_all=True)
+    for r in range(2):
+        p = int(b.q_pos[r])
+        np.testing.assert_allclose(h["block_scores"][r][1:p], d["all"][r][1:p], rtol=1e-13)
+        assert np.all(np.isnan(h["block_scores"][r][[0, p]]))
+        mid_top = ref_topk(d["all"][r][1:p], 3)
+        assert h["kept"][r].tolist() == sorted([0, p] + [1 + x for x in mid_top])
+
+
+def test_hisa_forced_blocks_and_external_kept():
+    b = workloads.hisa_decode(seed=4, B=2, L=4096, H=4, d=32, k=64, block=128, keep=4, n_needles=3)
+    h = oracle.hisa(b, B=128, keep=4, k=64)
+    for r in range(b.n_q):
+        kept = [x for x in h["kept"][r].tolist() if x >= 0]
+        assert kept[0] == 0 and kept[-1] == (int(b.q_pos[r])) // 128 and len(kept) == 6
+        assert kept == sorted(kept)
+    ext = oracle.hisa(b, B=128, keep=4, k=64, ext_kept=h["kept"])
+    assert np.array_equal(ext["idx"], h["idx"])
