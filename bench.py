@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA lightning indexer (score + top-k) on B200.
+
+One step = one call of the library's dense indexer top-k over one synthetic
+dense prefill sequence (T = L = 32768 causal, H = 64, d = 128, k = 2048):
+every query scores its whole causal prefix and keeps its top 2048 keys.
+The headline `value` is eligible (query, key) pairs per second, in Gpairs/s,
+summed over all ranks (each rank processes its own sequence: weak scaling,
+no collective on the data path).  Secondary entries (N = 1 only) time the
+other workloads of the same library: batched decode at 32K and 128K
+(us/step), PIVOT group-proxy prefill at 128K (Reuse and Refine) and HISA
+decode at 256K.
+
+Timing: W warm-up steps, then K steps each bracketed by CUDA events on the
+launching stream, a 256 MiB L2 flush between steps (outside the events),
+a barrier and a device synchronise on both sides of the timed region, and
+the max over ranks.  `--impl reference` times the fp64 CPU oracle instead
+(rank 0 only) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "indexer (score+top-k) Gpairs/s prefill"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SM_COUNT, FP32_LANES_PER_SM = 148, 128
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK, sm_max_mhz=1965.0), "fallback"
+
+
+# ----------------------------------------------------------------- ranks
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.gpu = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            self.gpu = None
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.gpu:
+            cmd += ["-i", self.gpu]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        self.out.seek(0)
+        rows = [r.split(",") for r in self.out.read().strip().splitlines() if r.count(",") >= 7]
+        os.unlink(self.out.name)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].strip() == "Active"})
+        loaded = [s for s in sm if mx and s >= 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------- timing
+
+class L2Flush:
+    def __init__(self, device, nbytes=256 << 20):
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def time_steps(step, n, flush):
+    """Device time (ms) of n steps, each between CUDA events on the current stream, L2 flushed before each."""
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in ev:
+        flush()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+# ------------------------------------------------------------ workloads
+
+class DenseTopk:
+    """Dense indexer top-k of a batch (prefill or decode) through the C ABI."""
+
+    def __init__(self, b, device):
+        import sparse_attention_indexer_04_b200 as dsa
+        self.dsa, self.b, self.k = dsa, b, int(b.params["k"])
+        self.lay = dsa.Layout.from_batch(b, device)
+        self.Q, self.K, self.W = b.Q.to(device), b.K.to(device), b.W.to(device)
+        self.idx = torch.empty(b.n_q, self.k, dtype=torch.int32, device=device)
+        self.ws = torch.empty(dsa.index_topk_workspace(self.lay, self.k), dtype=torch.uint8, device=device)
+        self.pairs = b.eligible_pairs()
+        self.device = device
+
+    def __call__(self):
+        self.dsa.index_topk(self.lay, self.Q, self.K, self.W, self.k, idx=self.idx, ws=self.ws)
+
+    def alg_bytes(self):
+        b = self.b
+        return b.K.numel() * 2 + b.Q.numel() * 2 + b.W.numel() * 4 + b.n_q * self.k * 4
+
+    def e2e(self, steps, flush):
+        """Same call from pinned host buffers: H2D of every input, the call, D2H of the indices, per step."""
+        b, dsa = self.b, self.dsa
+        hQ, hK, hW = b.Q.pin_memory(), b.K.pin_memory(), b.W.pin_memory()
+        hqo, hko, hpos = b.q_offsets.pin_memory(), b.k_offsets.pin_memory(), b.q_pos.pin_memory()
+        hidx = torch.empty(b.n_q, self.k, dtype=torch.int32).pin_memory()
+        lay = self.lay
+
+        def step():
+            self.Q.copy_(hQ, non_blocking=True)
+            self.K.copy_(hK, non_blocking=True)
+            self.W.copy_(hW, non_blocking=True)
+            lay.q_off.copy_(hqo, non_blocking=True)
+            lay.k_off.copy_(hko, non_blocking=True)
+            lay.q_pos.copy_(hpos, non_blocking=True)
+            dsa.index_topk(lay, self.Q, self.K, self.W, self.k, idx=self.idx, ws=self.ws)
+            hidx.copy_(self.idx, non_blocking=True)
+
+        for _ in range(2):
+            step()
+        ms = time_steps(step, steps, flush)
+        h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hW, hqo, hko, hpos))
+        return sum(ms) / steps, h2d, hidx.numel() * 4
+
+
+class Pivot:
+    def __init__(self, b, device, mode):
+        import sparse_attention_indexer_04_b200 as dsa
+        self.dsa, self.b, self.mode = dsa, b, mode
+        p = b.params
+        self.k, self.G, self.C = int(p["k"]), int(p["group"]), int(p["n_cand"])
+        self.lay = dsa.Layout.from_batch(b, device)
+        self.Q, self.K, self.W = b.Q.to(device), b.K.to(device), b.W.to(device)
+        self.idx = torch.empty(b.n_q, self.k, dtype=torch.int32, device=device)
+        self.ws = torch.empty(dsa.pivot_group_index_workspace(self.lay, self.k, self.G, self.C, mode),
+                              dtype=torch.uint8, device=device)
+
+    def __call__(self):
+        self.dsa.pivot_group_index(self.lay, self.Q, self.K, self.W, self.k, self.G, self.C, self.mode,
+                                   idx=self.idx, ws=self.ws)
+
+
+class Hisa:
+    def __init__(self, b, device):
+        import sparse_attention_indexer_04_b200 as dsa
+        self.dsa, self.b = dsa, b
+        p = b.params
+        self.k, self.B, self.keep = int(p["k"]), int(p["block"]), int(p["keep"])
+        self.lay = dsa.Layout.from_batch(b, device)
+        self.Q, self.K, self.W = b.Q.to(device), b.K.to(device), b.W.to(device)
+        self.pooled = dsa.hisa_pool_keys(self.lay, self.K, self.B)
+        self.idx = torch.empty(b.n_q, self.k, dtype=torch.int32, device=device)
+        self.ws = torch.empty(dsa.hisa_index_workspace(self.lay, self.k, self.B, self.keep), dtype=torch.uint8,
+                              device=device)
+
+    def __call__(self):
+        self.dsa.hisa_index(self.lay, self.Q, self.K, self.W, self.pooled, self.k, self.B, self.keep,
+                            idx=self.idx, ws=self.ws)
+
+
+def secondary(device, flush, steps):
+    out = {}
+
+    def run(name, make, extra):
+        try:
+            t0 = time.time()
+            step = make()
+            for _ in range(3):
+                step()
+            ms = time_steps(step, steps, flush)
+            r = {"us_per_step": round(1e3 * sum(ms) / steps, 2), "steps": steps, "setup_s": round(time.time() - t0, 1)}
+            r.update(extra(step, sum(ms) / steps))
+            out[name] = r
+            del step
+            torch.cuda.empty_cache()
+        except Exception as e:  # keep the headline line even if a secondary workload fails
+            out[name] = {"error": f"{type(e).__name__}: {e}"[:300]}
+
+    hbm = load_peaks()[0]["hbm_gbs"]
+
+    def dec_extra(step, ms):
+        gbs = step.alg_bytes() / (ms * 1e-3) / 1e9
+        return {"alg_bytes": step.alg_bytes(), "achieved_gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+
+    run("dense_decode_B16_L32768_mtp2", lambda: DenseTopk(workloads.dense_decode(seed=1), device), dec_extra)
+    run("dense_decode_B16_L131072_mtp2", lambda: DenseTopk(workloads.dense_decode(seed=1, L=131072), device),
+        dec_extra)
+    pv = workloads.pivot_prefill(seed=3)
+    dense_pairs = pv.eligible_pairs()
+    for mode, name in ((0, "reuse"), (1, "refine")):
+        run(f"pivot_prefill_T131072_G16_C8192_{name}", lambda m=mode: Pivot(pv, device, m),
+            lambda step, ms: {"dense_equiv_gpairs_s": round(dense_pairs / (ms * 1e-3) / 1e9, 2)})
+    del pv
+    run("hisa_decode_B4_L262144_keep64", lambda: Hisa(workloads.hisa_decode(seed=4), device), lambda s, ms: {})
+    return out
+
+
+# ------------------------------------------------------------ baselines
+
+def oracle_sample(b, k, budget_s=15.0, max_rows=64):
+    """Oracle dense top-k on a growing stratified row sample until ~budget_s of CPU time."""
+    import oracle
+    threads = oracle.default_threads()
+    n = 4
+    while True:
+        rows = workloads.stratified_rows(b.n_q, n_sample=n, head=1, tail=1)
+        pairs = sum(min(int(b.q_pos[r]) + 1, b.seq_lens()[0]) for r in rows)
+        t0 = time.perf_counter()
+        oracle.dense(b, rows=rows, k=k, threads=threads)
+        dt = time.perf_counter() - t0
+        if dt > budget_s / 3 or n >= max_rows:
+            return pairs, dt, threads, rows
+        n *= 2
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import oracle
+    b = workloads.dense_prefill(seed=2)
+    k = int(b.params["k"])
+    threads = oracle.default_threads()
+    rows = workloads.stratified_rows(b.n_q, n_sample=32, head=1, tail=1)
+    pairs = sum(int(b.q_pos[r]) + 1 for r in rows)
+    for _ in range(args.warmup):
+        oracle.dense(b, rows=rows[:2], k=k, threads=threads)
+    t = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.dense(b, rows=rows, k=k, threads=threads)
+        t.append(time.perf_counter() - t0)
+    sec = sum(t) / len(t)
+    value = pairs / sec / 1e9
+    sample = f"{len(rows)} stratified query rows of the 32K prefill ({pairs} pairs) per step"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Gpairs/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "dense_prefill_T32768_H64_d128_k2048", "T": 32768, "L": 32768, "H": 64, "d": 128,
+                   "k": 2048, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "Gpairs/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "Gpairs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+# ----------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--secondary-steps", type=int, default=5)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    world, rank, local = dist_setup()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import sparse_attention_indexer_04_b200 as dsa
+
+    peaks, peaks_src = load_peaks()
+    b = workloads.dense_prefill(seed=2 + 1000 * rank)
+    step = DenseTopk(b, device)
+    flush = L2Flush(device)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = dsa.launch_count()
+    with ClockSampler(device) as clk:
+        ms = time_steps(step, args.steps, flush)
+    launches = dsa.launch_count() - n0
+    barrier(world)
+    torch.cuda.synchronize()
+    total_ms = max_over_ranks(sum(ms), world)
+    ms_per_step = total_ms / args.steps
+    value = step.pairs * world / (ms_per_step * 1e-3) / 1e9
+
+    # ---- per-kernel times over a second pass of the same steps (events on the launching stream)
+    dsa.profile_enable(True)
+    time_steps(step, args.steps, flush)
+    prof = dsa.profile_read()
+    dsa.profile_enable(False)
+    dom, (dom_ms, dom_n) = max(prof.items(), key=lambda kv: kv[1][0])
+    flops_step = step.pairs * 2 * b.H * b.d
+    dom_ms_step = dom_ms / args.steps
+    if dom.startswith("score_simt"):
+        clk_max = peaks.get("sm_max_mhz", 1965.0)
+        peak = SM_COUNT * FP32_LANES_PER_SM * 2 * clk_max * 1e6 / 1e12
+        roof = {"bound": "alu", "unit": "TFLOP/s", "peak_basis": f"fp32 FMA: {SM_COUNT} SMs x "
+                f"{FP32_LANES_PER_SM} lanes x 2 flop x {clk_max:.0f} MHz"}
+    else:
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_basis": f"bf16 dense, {peaks_src}"}
+    achieved = flops_step / (dom_ms_step * 1e-3) / 1e12
+    roof.update({"kernel": dom, "achieved": round(achieved, 3), "peak": round(peak, 1),
+                 "frac": round(achieved / peak, 4), "traffic": None, "launches_per_step": dom_n / args.steps,
+                 "kernel_ms_per_step": round(dom_ms_step, 3),
+                 "kernel_share": round(dom_ms / sum(v[0] for v in prof.values()), 4),
+                 "per_kernel_ms_per_step": {k: round(v[0] / args.steps, 3) for k, v in prof.items()}})
+
+    e2e_ms, h2d, d2h = step.e2e(max(2, args.steps // 2), flush)
+    e2e = {"value": step.pairs * world / (max_over_ranks(e2e_ms, world) * 1e-3) / 1e9, "unit": "Gpairs/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    sec = {}
+    if rank == 0 and world == 1:
+        if not args.no_secondary:
+            del step
+            torch.cuda.empty_cache()
+            sec = secondary(device, flush, args.secondary_steps)
+        pairs, dt, threads, rows = oracle_sample(b, int(b.params["k"]))
+        cpu = {"value": pairs / dt / 1e9, "unit": "Gpairs/s", "cores": threads, "kind": "oracle",
+               "sample": f"{len(rows)} stratified query rows of the 32K prefill ({pairs} pairs), {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "Gpairs/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "dense_prefill_T32768_H64_d128_k2048", "T": 32768, "L": 32768, "H": 64,
+                       "d": 128, "k": 2048, "global_batch": world, "seq_len": 32768,
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "flushed between timed steps (256 MiB write)",
+                       "pairs_per_step_per_gpu": step_pairs(b)},
+            "clocks": clk.summary(), "e2e": e2e, "gpu_launches": launches, "roofline": roof,
+            "cpu_baseline": cpu, "secondary": sec, "peaks": peaks_src,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def step_pairs(b):
+    return b.eligible_pairs()
+
+
+if __name__ == "__main__":
+    main()

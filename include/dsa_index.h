@@ -1,0 +1,201 @@
+/*
+ * dsa_index.h — C ABI of libdsaidx, a B200 (sm_100a) library for the
+ * DeepSeek Sparse Attention (DSA) lightning indexer and two scan-reducing
+ * variants of it.
+ *
+ * What is computed.  For query t of a sequence (H heads of dimension d, a
+ * weight per head) and key s of the same sequence (one key per token, shared
+ * by every head) the indexer score is
+ *
+ *        I[t,s] = sum_h  w[t,h] * max(0, q[t,h] . k[s])
+ *
+ * and the indexer keeps, for every query, the k keys with the highest score
+ * among its causal prefix.  The pages this library follows describe the
+ * indexer in words only ("Multi-layer Indexer: overlapping selection and
+ * attention in DeepSeek Sparse Attention", abstract: the indexer scores the
+ * whole cache and keeps the k = 2048 best tokens; "PIVOT: Efficient
+ * Query-Group Indexing for Token-Level Sparse Attention", abstract: each
+ * query scores every preceding token).  The formula is DeepSeek-V3.2's.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  Data types and layouts (row-major, densely packed, device memory):
+ *    Q  [n_q, H, d]  bf16 (passed as const void*), rows 16-byte aligned
+ *    K  [n_k, d]     bf16, rows 16-byte aligned
+ *    W  [n_q, H]     fp32
+ *  Sequences.  A batch holds B sequences.  Sequence b owns query rows
+ *  [q_offsets[b], q_offsets[b+1]) and key rows [k_offsets[b],
+ *  k_offsets[b+1]).  q_pos[t] is query t's position inside its sequence.
+ *  Causality.  Query t may select key s (a sequence-local index) when
+ *  s <= q_pos[t] and s < L_b (the key count of its sequence): the query's
+ *  own token is part of its prefix.  A negative position leaves the row
+ *  empty.
+ *  Ranking.  Higher score first; equal scores go to the lower key index.
+ *  A score of -0 ranks as +0.
+ *  Output rows.  Every index row holds min(k, #eligible) sequence-local key
+ *  indices in ASCENDING index order, then -1 padding up to k.  Optional
+ *  score outputs hold the fp32 score of each returned index (NaN padding).
+ *  Supported shapes.  H in {1..64} with H*d*2 a multiple of 16; d in
+ *  {32, 64, 128}; 1 <= k <= 16384; per-sequence key count < 2^31.
+ *  Otherwise DSA_ERR_UNSUPPORTED.
+ *  Ownership.  The caller owns every buffer: inputs, outputs and the
+ *  workspace.  The library allocates no device memory, never synchronises
+ *  the stream (dsa_device_check and dsa_profile_read excepted) and keeps no
+ *  per-call state.
+ *  Workspace.  Every call that takes `ws` needs at least the bytes its
+ *  *_workspace function returns for the same arguments, 256-byte aligned.
+ *  Its first 256 bytes hold a device status word: kernels that detect a
+ *  problem (a bounded wait that ran out) record it there and return early;
+ *  dsa_device_check reads it.  Calls overlapping on the GPU need distinct
+ *  workspaces.
+ *  Streams.  `stream` is a cudaStream_t (NULL = legacy default stream).  All
+ *  work is enqueued on it; results are ready when the stream reaches them.
+ *  Errors.  Argument checks run on the host before anything is enqueued and
+ *  return DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED / DSA_ERR_WORKSPACE with
+ *  nothing launched.  A failed launch returns DSA_ERR_CUDA.  Faults that
+ *  happen later on the device surface at the caller's next synchronisation.
+ *  Non-finite inputs give undefined rankings.
+ *  Thread safety.  Entry points may be called from several host threads
+ *  at once given distinct workspaces.
+ */
+#ifndef DSA_INDEX_H
+#define DSA_INDEX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dsa_status {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad offsets, misalignment */
+    DSA_ERR_UNSUPPORTED = 2,   /* shape outside the supported set */
+    DSA_ERR_WORKSPACE = 3,     /* workspace missing, too small or misaligned */
+    DSA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    DSA_ERR_DEVICE_CHECK = 5   /* a kernel recorded an error in the workspace status word */
+} dsa_status;
+
+/* A ragged batch of sequences.  The device arrays are read by the kernels;
+ * the host copies (same values) size grids and workspaces without a
+ * device-to-host copy.  All pointers stay owned by the caller. */
+typedef struct dsa_batch {
+    int32_t num_seqs;              /* B >= 1 */
+    int32_t num_heads;             /* H */
+    int32_t head_dim;              /* d */
+    int32_t num_queries;           /* n_q = q_offsets[B] (may be 0) */
+    int32_t num_keys;              /* n_k = k_offsets[B] */
+    const int32_t* q_offsets;      /* device [B+1], non-decreasing, q_offsets[0] = 0 */
+    const int32_t* k_offsets;      /* device [B+1], non-decreasing, k_offsets[0] = 0 */
+    const int32_t* q_pos;          /* device [n_q] */
+    const int32_t* q_offsets_host; /* host   [B+1] */
+    const int32_t* k_offsets_host; /* host   [B+1] */
+} dsa_batch;
+
+/* Human-readable name of a status code (static storage). */
+const char* dsa_status_string(dsa_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t dsa_version(void);
+
+/* --------------------------------------------------------------------
+ * Dense indexer scores (debug / reference view of the contraction).
+ * S [n_q, ld_s] fp32: S[t][s] = I[t,s] for eligible s, -inf for every other
+ * s < ld_s.  ld_s >= the longest sequence's key count.  The full score matrix
+ * is written, so this call is for inspection, not the hot path.
+ * Source: the indexer score of the MLI and PIVOT abstracts.
+ */
+size_t dsa_index_scores_workspace(const dsa_batch* batch);
+dsa_status dsa_index_scores(const dsa_batch* batch, const void* Q, const void* K, const float* W,
+                            float* S, int64_t ld_s, void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------
+ * Dense indexer top-k: for every query, the k best eligible keys.
+ * idx [n_q, k] int32; scores [n_q, k] fp32 or NULL.
+ * Source: MLI abstract (score the whole cache, keep k = 2048); PIVOT
+ * abstract (every preceding token is scored, O(L^2) per layer in prefill).
+ * Prefill (one query per position) and batched decode (a few MTP queries
+ * per sequence at its end) are the same call with different q_pos.
+ */
+size_t dsa_index_topk_workspace(const dsa_batch* batch, int32_t k);
+dsa_status dsa_index_topk(const dsa_batch* batch, const void* Q, const void* K, const float* W,
+                          int32_t k, int32_t* idx, float* scores, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* --------------------------------------------------------------------
+ * PIVOT group-proxy indexing ("PIVOT: Efficient Query-Group Indexing for
+ * Token-Level Sparse Attention", abstract).
+ * Groups: inside each sequence, consecutive runs of `group` query rows (the
+ * last run may be shorter); in decode pass group >= the MTP query count so
+ * that a group is one MTP step.  Groups are numbered in sequence order;
+ * pivot_num_groups returns their count.
+ * Proxy: q_bar = bf16(mean of the group's q, rounded to nearest even),
+ * w_bar = mean of the group's w.  The proxy scans its sequence's keys
+ * s <= max q_pos of the group and keeps the n_cand best (the candidate set).
+ * mode 0 (Reuse):  query t takes the k best candidates by proxy score among
+ *                  candidates s <= q_pos[t].
+ * mode 1 (Refine): query t scores the candidates s <= q_pos[t] with its own
+ *                  q and w and takes its own top k.
+ * idx [n_q, k] int32 (rows in query order); cand [n_groups, n_cand] int32 or
+ * NULL (ascending, -1 padded).  Requires k <= n_cand <= 16384, 1 <= group <= 64.
+ */
+int32_t pivot_num_groups(const dsa_batch* batch, int32_t group);
+size_t pivot_group_index_workspace(const dsa_batch* batch, int32_t k, int32_t group,
+                                   int32_t n_cand, int32_t mode);
+dsa_status pivot_group_index(const dsa_batch* batch, const void* Q, const void* K, const float* W,
+                             int32_t k, int32_t group, int32_t n_cand, int32_t mode, int32_t* idx,
+                             int32_t* cand, void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------
+ * HISA hierarchical indexing ("HISA: Efficient Hierarchical Indexing for
+ * Fine-Grained Sparse Attention", abstract).
+ * hisa_pool_keys: pooled [n_blocks, d] fp32, the mean of the keys of each
+ * block of `block` tokens (the last block of a sequence may be partial);
+ * blocks of all sequences stacked in order, hisa_num_blocks of them.
+ * hisa_index: for query t, with last = q_pos[t] / block (clamped to the
+ * sequence), the blocks strictly between block 0 and `last` are scored with
+ * the indexer formula against their pooled key; block 0, block `last` and the
+ * `keep` best middle blocks are kept; the indexer then ranks every eligible
+ * token of the kept blocks and returns its top k.
+ * idx [n_q, k]; kept [n_q, keep+2] int32 or NULL (ascending, -1 padded).
+ * Requires block in {64, 128, 256}, 1 <= keep <= 256.
+ */
+int64_t hisa_num_blocks(const dsa_batch* batch, int32_t block);
+dsa_status hisa_pool_keys(const dsa_batch* batch, const void* K, int32_t block, float* pooled,
+                          void* stream);
+size_t hisa_index_workspace(const dsa_batch* batch, int32_t k, int32_t block, int32_t keep);
+dsa_status hisa_index(const dsa_batch* batch, const void* Q, const void* K, const float* W,
+                      const float* pooled, int32_t k, int32_t block, int32_t keep, int32_t* idx,
+                      int32_t* kept, void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------
+ * Reads the workspace status word written by the kernels of earlier calls
+ * on `stream` (synchronises the stream).  Returns DSA_OK when no kernel
+ * recorded a problem, else DSA_ERR_DEVICE_CHECK and, if `detail` is not
+ * NULL, the recorded code (see the kernels' documentation).  Clears it.
+ */
+dsa_status dsa_device_check(void* ws, void* stream, uint32_t* detail);
+
+/* --------------------------------------------------------------------
+ * Launch accounting and kernel timing, for benchmarks (not part of the
+ * indexer; no counterpart on the pages).  The only process-wide state of
+ * the library.
+ * dsa_launch_count: kernels launched by this library since load.
+ * dsa_profile_enable(1): from then on every launch is bracketed by two CUDA
+ * events recorded on its own stream.  dsa_profile_read synchronises those
+ * events, adds up per kernel kind (index 0 .. n-1, names from
+ * dsa_profile_kind_name) the elapsed milliseconds and launch counts into
+ * ms[] / launches[] (each `cap` long, either may be NULL), forgets them, and
+ * returns the number of kinds (or -1 if an event failed).
+ */
+void dsa_profile_enable(int32_t on);
+uint64_t dsa_launch_count(void);
+const char* dsa_profile_kind_name(int32_t kind);
+int32_t dsa_profile_read(float* ms, int32_t* launches, int32_t cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_INDEX_H */

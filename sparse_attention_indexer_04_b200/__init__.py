@@ -1,0 +1,260 @@
+"""Python binding of libdsaidx, the B200 DSA lightning-indexer library.
+
+Argument marshalling only: every step of the indexer runs in the library's
+CUDA kernels.  Tensors are torch CUDA tensors (PyTorch supplies device
+memory and the current stream); the library itself allocates nothing, so
+outputs and workspaces are allocated here with torch and handed over as raw
+pointers.  There is no CPU fallback: importing this package fails loudly
+when the compiled library is missing.
+
+Entry points mirror include/dsa_index.h:
+  index_scores, index_topk, pivot_group_index, hisa_pool_keys, hisa_index,
+  device_check, plus the *_workspace size queries.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsaidx.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python sparse_attention_indexer_04_b200/build.py` "
+                      "(or __graft_entry__.build()); there is no fallback path")
+_lib = ctypes.CDLL(LIB_PATH)
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "workspace", 4: "CUDA error",
+          5: "device check"}
+REUSE, REFINE = 0, 1
+
+
+class DsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib.dsa_status_string(status).decode()} (status {status})")
+
+
+class _Batch(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("num_queries", ctypes.c_int32), ("num_keys", ctypes.c_int32),
+                ("q_offsets", ctypes.c_void_p), ("k_offsets", ctypes.c_void_p), ("q_pos", ctypes.c_void_p),
+                ("q_offsets_host", ctypes.c_void_p), ("k_offsets_host", ctypes.c_void_p)]
+
+
+_P = ctypes.c_void_p
+_B = ctypes.POINTER(_Batch)
+_I32, _I64, _SZ = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+
+
+def _sig(name, res, *args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = list(args)
+    return f
+
+
+_sig("dsa_status_string", ctypes.c_char_p, ctypes.c_int)
+_sig("dsa_version", _I32)
+_sig("dsa_index_scores_workspace", _SZ, _B)
+_sig("dsa_index_scores", ctypes.c_int, _B, _P, _P, _P, _P, _I64, _P, _SZ, _P)
+_sig("dsa_index_topk_workspace", _SZ, _B, _I32)
+_sig("dsa_index_topk", ctypes.c_int, _B, _P, _P, _P, _I32, _P, _P, _P, _SZ, _P)
+_sig("pivot_num_groups", _I32, _B, _I32)
+_sig("pivot_group_index_workspace", _SZ, _B, _I32, _I32, _I32, _I32)
+_sig("pivot_group_index", ctypes.c_int, _B, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _SZ, _P)
+_sig("hisa_num_blocks", _I64, _B, _I32)
+_sig("hisa_pool_keys", ctypes.c_int, _B, _P, _I32, _P, _P)
+_sig("hisa_index_workspace", _SZ, _B, _I32, _I32, _I32)
+_sig("hisa_index", ctypes.c_int, _B, _P, _P, _P, _P, _I32, _I32, _I32, _P, _P, _P, _SZ, _P)
+_sig("dsa_device_check", ctypes.c_int, _P, _P, ctypes.POINTER(ctypes.c_uint32))
+_sig("dsa_profile_enable", None, _I32)
+_sig("dsa_launch_count", ctypes.c_uint64)
+_sig("dsa_profile_kind_name", ctypes.c_char_p, _I32)
+_sig("dsa_profile_read", _I32, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32), _I32)
+
+
+def library():
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise DsaError(status, where)
+
+
+class Layout:
+    """Sequence layout of a batch: offsets and positions on the device plus host copies.
+
+    q_offsets / k_offsets: [B+1] row offsets of each sequence's queries / keys;
+    q_pos: [n_q] sequence-local position of each query.
+    """
+
+    def __init__(self, q_offsets, k_offsets, q_pos, num_heads: int, head_dim: int, device="cuda"):
+        self.q_off_host = torch.as_tensor(q_offsets, dtype=torch.int32).cpu().contiguous()
+        self.k_off_host = torch.as_tensor(k_offsets, dtype=torch.int32).cpu().contiguous()
+        self.q_off = self.q_off_host.to(device)
+        self.k_off = self.k_off_host.to(device)
+        self.q_pos = torch.as_tensor(q_pos, dtype=torch.int32).to(device).contiguous()
+        self.num_heads, self.head_dim = int(num_heads), int(head_dim)
+        self.device = torch.device(device)
+        self.c = _Batch(int(self.q_off_host.numel() - 1), self.num_heads, self.head_dim,
+                        int(self.q_off_host[-1]), int(self.k_off_host[-1]),
+                        self.q_off.data_ptr(), self.k_off.data_ptr(),
+                        self.q_pos.data_ptr() if self.q_pos.numel() else None,
+                        self.q_off_host.data_ptr(), self.k_off_host.data_ptr())
+
+    @classmethod
+    def from_batch(cls, b, device="cuda"):
+        return cls(b.q_offsets, b.k_offsets, b.q_pos, b.H, b.d, device)
+
+    @property
+    def num_queries(self):
+        return self.c.num_queries
+
+    @property
+    def max_keys(self):
+        ko = self.k_off_host
+        return int((ko[1:] - ko[:-1]).max()) if ko.numel() > 1 else 0
+
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+def _workspace(nbytes: int, device, ws=None):
+    if ws is not None:
+        return ws
+    # 256-byte aligned: torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def _bytes(ws):
+    return ctypes.c_size_t(ws.numel() * ws.element_size())
+
+
+# ------------------------------------------------------------------- dense
+
+def index_scores_workspace(layout: Layout) -> int:
+    return int(_lib.dsa_index_scores_workspace(layout.ref()))
+
+
+def index_scores(layout: Layout, Q, K, W, S=None, ws=None, stream=None):
+    """Dense indexer scores: S [n_q, ld] fp32, -inf where the key is not eligible."""
+    if S is None:
+        S = torch.empty(layout.num_queries, max(layout.max_keys, 1), dtype=torch.float32, device=layout.device)
+    ws = _workspace(index_scores_workspace(layout), layout.device, ws)
+    _check(_lib.dsa_index_scores(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), _ptr(S), S.stride(0), _ptr(ws),
+                                 _bytes(ws), _stream(stream)), "dsa_index_scores")
+    return S
+
+
+def index_topk_workspace(layout: Layout, k: int) -> int:
+    return int(_lib.dsa_index_topk_workspace(layout.ref(), k))
+
+
+def index_topk(layout: Layout, Q, K, W, k: int, idx=None, scores=None, want_scores=False, ws=None, stream=None):
+    """Dense indexer top-k: idx [n_q, k] int32 (ascending, -1 padded), optional scores [n_q, k]."""
+    if idx is None:
+        idx = torch.empty(layout.num_queries, k, dtype=torch.int32, device=layout.device)
+    if want_scores and scores is None:
+        scores = torch.empty(layout.num_queries, k, dtype=torch.float32, device=layout.device)
+    ws = _workspace(index_topk_workspace(layout, k), layout.device, ws)
+    _check(_lib.dsa_index_topk(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), k, _ptr(idx), _ptr(scores), _ptr(ws),
+                               _bytes(ws), _stream(stream)), "dsa_index_topk")
+    return (idx, scores) if want_scores else idx
+
+
+# ------------------------------------------------------------------- PIVOT
+
+def pivot_num_groups(layout: Layout, group: int) -> int:
+    return int(_lib.pivot_num_groups(layout.ref(), group))
+
+
+def pivot_group_index_workspace(layout: Layout, k: int, group: int, n_cand: int, mode: int) -> int:
+    return int(_lib.pivot_group_index_workspace(layout.ref(), k, group, n_cand, mode))
+
+
+def pivot_group_index(layout: Layout, Q, K, W, k: int, group: int, n_cand: int, mode: int, idx=None, cand=None,
+                      want_cand=False, ws=None, stream=None):
+    """PIVOT Reuse (mode 0) / Refine (mode 1): idx [n_q, k]; optional cand [n_groups, n_cand]."""
+    if idx is None:
+        idx = torch.empty(layout.num_queries, k, dtype=torch.int32, device=layout.device)
+    if want_cand and cand is None:
+        cand = torch.empty(max(pivot_num_groups(layout, group), 0), n_cand, dtype=torch.int32, device=layout.device)
+    ws = _workspace(pivot_group_index_workspace(layout, k, group, n_cand, mode), layout.device, ws)
+    _check(_lib.pivot_group_index(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), k, group, n_cand, mode, _ptr(idx),
+                                  _ptr(cand), _ptr(ws), _bytes(ws), _stream(stream)), "pivot_group_index")
+    return (idx, cand) if want_cand else idx
+
+
+# -------------------------------------------------------------------- HISA
+
+def hisa_num_blocks(layout: Layout, block: int) -> int:
+    return int(_lib.hisa_num_blocks(layout.ref(), block))
+
+
+def hisa_pool_keys(layout: Layout, K, block: int, pooled=None, stream=None):
+    """Mean-pooled block keys [n_blocks, d] fp32."""
+    if pooled is None:
+        pooled = torch.empty(max(hisa_num_blocks(layout, block), 0), layout.head_dim, dtype=torch.float32,
+                             device=layout.device)
+    _check(_lib.hisa_pool_keys(layout.ref(), _ptr(K), block, _ptr(pooled), _stream(stream)), "hisa_pool_keys")
+    return pooled
+
+
+def hisa_index_workspace(layout: Layout, k: int, block: int, keep: int) -> int:
+    return int(_lib.hisa_index_workspace(layout.ref(), k, block, keep))
+
+
+def hisa_index(layout: Layout, Q, K, W, pooled, k: int, block: int, keep: int, idx=None, kept=None,
+               want_kept=False, ws=None, stream=None):
+    """HISA top-k: idx [n_q, k]; optional kept [n_q, keep+2] block lists."""
+    if idx is None:
+        idx = torch.empty(layout.num_queries, k, dtype=torch.int32, device=layout.device)
+    if want_kept and kept is None:
+        kept = torch.empty(layout.num_queries, keep + 2, dtype=torch.int32, device=layout.device)
+    ws = _workspace(hisa_index_workspace(layout, k, block, keep), layout.device, ws)
+    _check(_lib.hisa_index(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), _ptr(pooled), k, block, keep, _ptr(idx),
+                           _ptr(kept), _ptr(ws), _bytes(ws), _stream(stream)), "hisa_index")
+    return (idx, kept) if want_kept else idx
+
+
+def launch_count() -> int:
+    """Kernels this library has launched since it was loaded."""
+    return int(_lib.dsa_launch_count())
+
+
+def profile_enable(on: bool = True):
+    """Bracket every later launch with CUDA events on its own stream (see profile_read)."""
+    _lib.dsa_profile_enable(1 if on else 0)
+
+
+def profile_read():
+    """{kernel kind: (total ms, launches)} since the last read; synchronises the recorded events."""
+    cap = 32
+    ms = (ctypes.c_float * cap)()
+    n = (ctypes.c_int32 * cap)()
+    kinds = _lib.dsa_profile_read(ms, n, cap)
+    if kinds < 0:
+        raise DsaError(4, "dsa_profile_read")
+    return {_lib.dsa_profile_kind_name(i).decode(): (float(ms[i]), int(n[i])) for i in range(kinds) if n[i]}
+
+
+def device_check(ws, stream=None) -> int:
+    """Status word recorded by kernels in a workspace (0 = none); synchronises the stream."""
+    detail = ctypes.c_uint32(0)
+    st = _lib.dsa_device_check(_ptr(ws), _stream(stream), ctypes.byref(detail))
+    if st not in (0, 5):
+        raise DsaError(st, "dsa_device_check")
+    return int(detail.value) if st == 5 else 0

@@ -1,0 +1,592 @@
+// libdsaidx C ABI: argument checks, workspace layout and kernel launches.
+// Declarations and the contract of every entry point: include/dsa_index.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/dsa_index.h"
+#include "common.cuh"
+#include "score_simt.cuh"
+#include "select.cuh"
+#include "setup.cuh"
+
+using namespace dsa;
+
+namespace {
+
+constexpr int32_t kMaxK = 16384;
+constexpr int32_t kMaxCand = 16384;
+constexpr size_t kScoreBudget = size_t(256) << 20;   // bytes of materialised score rows per launch
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Sequential carve-out of a workspace; a dry run (base == nullptr) sizes it.
+struct Carver {
+    char* base;
+    size_t off = kStatusBytes;
+    template <typename T>
+    T* take(size_t count)
+    {
+        T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+        off = align256(off + count * sizeof(T));
+        return p;
+    }
+};
+
+bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+bool heads_ok(int h) { return h >= 1 && h <= 64 && (h & (h - 1)) == 0; }
+
+struct HostInfo {
+    int32_t max_q = 0;   // longest query run of a sequence
+    int32_t max_k = 0;   // longest key run of a sequence
+};
+
+dsa_status check_batch(const dsa_batch* b, HostInfo* info)
+{
+    if (!b) return DSA_ERR_INVALID_ARG;
+    if (b->num_seqs < 1 || b->num_queries < 0 || b->num_keys < 0) return DSA_ERR_INVALID_ARG;
+    if (!heads_ok(b->num_heads) || !head_dim_ok(b->head_dim)) return DSA_ERR_UNSUPPORTED;
+    if (!b->q_offsets || !b->k_offsets || !b->q_offsets_host || !b->k_offsets_host)
+        return DSA_ERR_INVALID_ARG;
+    if (b->num_queries > 0 && !b->q_pos) return DSA_ERR_INVALID_ARG;
+    const int32_t* qo = b->q_offsets_host;
+    const int32_t* ko = b->k_offsets_host;
+    if (qo[0] != 0 || ko[0] != 0) return DSA_ERR_INVALID_ARG;
+    for (int i = 0; i < b->num_seqs; ++i) {
+        if (qo[i + 1] < qo[i] || ko[i + 1] < ko[i]) return DSA_ERR_INVALID_ARG;
+        info->max_q = std::max(info->max_q, qo[i + 1] - qo[i]);
+        info->max_k = std::max(info->max_k, ko[i + 1] - ko[i]);
+    }
+    if (qo[b->num_seqs] != b->num_queries || ko[b->num_seqs] != b->num_keys) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+}
+
+dsa_status check_tensors(const dsa_batch* b, const void* Q, const void* K, const float* W)
+{
+    if (b->num_queries > 0 && (!Q || !W)) return DSA_ERR_INVALID_ARG;
+    if (b->num_keys > 0 && !K) return DSA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K)) & 15) return DSA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(W) & 3) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+}
+
+dsa_status check_ws(void* ws, size_t ws_bytes, size_t need)
+{
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255)) return DSA_ERR_WORKSPACE;
+    return DSA_OK;
+}
+
+dsa_status launched()
+{
+    return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------- profiling
+// Kernel kinds timed by the optional profiler (dsa_profile_*).
+enum ProfKind : int32_t { kProfSetup = 0, kProfScoreSimt, kProfSelect, kProfPool, kProfProxy, kProfKinds };
+const char* const kProfNames[kProfKinds] = {"setup", "score_simt", "select_topk", "hisa_pool", "pivot_proxy"};
+
+struct ProfRec {
+    int32_t kind;
+    cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+std::atomic<bool> g_prof_on{false};
+std::vector<ProfRec> g_prof;
+std::atomic<uint64_t> g_launches{0};
+
+#define DSA_LAUNCH(kind, st, ...)      \
+    do {                               \
+        LaunchScope _ls((kind), (st)); \
+        __VA_ARGS__;                   \
+    } while (0)
+
+// Counts one kernel launch; when profiling is on, brackets it with events on its stream.
+struct LaunchScope {
+    int32_t kind;
+    cudaStream_t st;
+    cudaEvent_t start = nullptr;
+    LaunchScope(int32_t k, cudaStream_t s) : kind(k), st(s)
+    {
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        if (g_prof_on.load(std::memory_order_relaxed) && cudaEventCreate(&start) == cudaSuccess)
+            cudaEventRecord(start, st);
+    }
+    ~LaunchScope()
+    {
+        if (!start) return;
+        cudaEvent_t stop;
+        if (cudaEventCreate(&stop) != cudaSuccess) { cudaEventDestroy(start); return; }
+        cudaEventRecord(stop, st);
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        g_prof.push_back(ProfRec{kind, start, stop});
+    }
+};
+
+int64_t score_ld(int32_t cols) { return std::max<int64_t>(4, (cols + 3) & ~3); }
+
+int32_t chunk_rows(int32_t n_rows, int64_t ld)
+{
+    const int64_t per = ld * int64_t(sizeof(float));
+    return (int32_t)std::max<int64_t>(1, std::min<int64_t>(n_rows, int64_t(kScoreBudget) / per));
+}
+
+// ------------------------------------------------------------ launchers
+
+template <typename KT>
+dsa_status launch_score(const RowDesc* rows, int32_t n_rows, int32_t max_cols, const ColMap& map,
+                        const void* Q, const float* W, int H, int D, const KT* K, const int32_t* k_base,
+                        float* S, int64_t ld_s, int32_t fill, cudaStream_t st)
+{
+    if (n_rows <= 0) return DSA_OK;
+    const int32_t cols = std::max(max_cols, fill);
+    if (cols <= 0) return DSA_OK;
+    ScoreArgs a{};
+    a.rows = rows; a.n_rows = n_rows; a.H = H; a.map = map;
+    a.Q = reinterpret_cast<const __nv_bfloat16*>(Q); a.W = W; a.K = K; a.k_base = k_base;
+    a.S = S; a.ld_s = ld_s; a.fill = fill;
+    const dim3 grid(n_rows, (cols + kSimtCols - 1) / kSimtCols);
+    const size_t smem = size_t(H) * D * sizeof(float) + size_t(H) * sizeof(float);
+    switch (D) {
+    case 32: DSA_LAUNCH(kProfScoreSimt, st, score_simt_kernel<32, KT><<<grid, kSimtCols, smem, st>>>(a)); break;
+    case 64: DSA_LAUNCH(kProfScoreSimt, st, score_simt_kernel<64, KT><<<grid, kSimtCols, smem, st>>>(a)); break;
+    default: DSA_LAUNCH(kProfScoreSimt, st, score_simt_kernel<128, KT><<<grid, kSimtCols, smem, st>>>(a)); break;
+    }
+    return launched();
+}
+
+dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, int32_t k, const ColMap& map,
+                         const float* S, int64_t ld_s, bool src_from_list, int32_t* out_idx, int64_t ld_idx,
+                         float* out_score, int64_t ld_score, cudaStream_t st)
+{
+    if (n_rows <= 0) return DSA_OK;
+    SelectArgs a{};
+    a.rows = rows; a.n_rows = n_rows; a.k = k; a.map = map; a.S = S; a.ld_s = ld_s;
+    a.src_from_list = src_from_list ? 1 : 0;
+    a.out_idx = out_idx; a.ld_idx = ld_idx; a.out_score = out_score; a.ld_score = ld_score;
+    if (max_cols <= kSelectSmemKeys) {
+        const size_t smem = size_t(std::max(max_cols, 1)) * sizeof(uint32_t);
+        if (cudaFuncSetAttribute(select_topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(kSelectSmemKeys * sizeof(uint32_t))) != cudaSuccess)
+            return DSA_ERR_CUDA;
+        DSA_LAUNCH(kProfSelect, st, select_topk_kernel<true><<<n_rows, kSelectThreads, smem, st>>>(a));
+    } else {
+        DSA_LAUNCH(kProfSelect, st, select_topk_kernel<false><<<n_rows, kSelectThreads, 0, st>>>(a));
+    }
+    return launched();
+}
+
+// Score then select, in row chunks that fit the score buffer.
+template <typename KT>
+dsa_status score_and_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, const ColMap& map,
+                            const void* Q, const float* W, int H, int D, const KT* K, const int32_t* k_base,
+                            float* Sbuf, int32_t k, int32_t* idx, int64_t ld_idx, float* scores,
+                            cudaStream_t st)
+{
+    const int64_t ld = score_ld(max_cols);
+    const int32_t chunk = chunk_rows(n_rows, ld);
+    for (int32_t r0 = 0; r0 < n_rows; r0 += chunk) {
+        const int32_t nr = std::min(chunk, n_rows - r0);
+        dsa_status s = launch_score<KT>(rows + r0, nr, max_cols, map, Q, W, H, D, K, k_base, Sbuf, ld, 0, st);
+        if (s != DSA_OK) return s;
+        s = launch_select(rows + r0, nr, max_cols, k, map, Sbuf, ld, false, idx + int64_t(r0) * ld_idx, ld_idx,
+                          scores ? scores + int64_t(r0) * ld_idx : nullptr, ld_idx, st);
+        if (s != DSA_OK) return s;
+    }
+    return DSA_OK;
+}
+
+ColMap identity_map(int32_t offset = 0)
+{
+    ColMap m{};
+    m.kind = kMapIdentity;
+    m.offset = offset;
+    return m;
+}
+
+// ------------------------------------------------------- workspace plans
+
+struct DensePlan {
+    RowDesc* rows;
+    float* S;
+};
+
+size_t dense_plan(char* base, const dsa_batch* b, const HostInfo& hi, bool scores_only, DensePlan* p)
+{
+    Carver c{base};
+    p->rows = c.take<RowDesc>(std::max(1, b->num_queries));
+    if (!scores_only) {
+        const int64_t ld = score_ld(hi.max_k);
+        p->S = c.take<float>(size_t(chunk_rows(std::max(1, b->num_queries), ld)) * ld);
+    }
+    return c.off;
+}
+
+struct PivotPlan {
+    int32_t* group_base;
+    GroupDesc* groups;
+    RowDesc* proxy_rows;
+    RowDesc* query_rows;
+    __nv_bfloat16* Qp;
+    float* Wp;
+    int32_t* cand;
+    float* cand_score;
+    float* S;
+};
+
+int32_t count_groups(const dsa_batch* b, int32_t G)
+{
+    int64_t n = 0;
+    for (int i = 0; i < b->num_seqs; ++i)
+        n += (b->q_offsets_host[i + 1] - b->q_offsets_host[i] + G - 1) / G;
+    return (int32_t)n;
+}
+
+size_t pivot_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t G, int32_t C, PivotPlan* p)
+{
+    Carver c{base};
+    const int32_t ng = std::max(1, count_groups(b, G));
+    p->group_base = c.take<int32_t>(b->num_seqs + 1);
+    p->groups = c.take<GroupDesc>(ng);
+    p->proxy_rows = c.take<RowDesc>(ng);
+    p->query_rows = c.take<RowDesc>(std::max(1, b->num_queries));
+    p->Qp = c.take<__nv_bfloat16>(size_t(ng) * b->num_heads * b->head_dim);
+    p->Wp = c.take<float>(size_t(ng) * b->num_heads);
+    p->cand = c.take<int32_t>(size_t(ng) * C);
+    p->cand_score = c.take<float>(size_t(ng) * C);
+    const int64_t ld_scan = score_ld(hi.max_k), ld_ref = score_ld(C);
+    const size_t s_scan = size_t(chunk_rows(ng, ld_scan)) * ld_scan;
+    const size_t s_ref = size_t(chunk_rows(std::max(1, b->num_queries), ld_ref)) * ld_ref;
+    p->S = c.take<float>(std::max(s_scan, s_ref));
+    return c.off;
+}
+
+struct HisaPlan {
+    int32_t* block_base;
+    RowDesc* block_rows;
+    RowDesc* token_rows;
+    int32_t* mid;
+    int32_t* kept;
+    float* S;
+};
+
+size_t hisa_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t B, int32_t keep, HisaPlan* p)
+{
+    Carver c{base};
+    const int32_t nq = std::max(1, b->num_queries);
+    p->block_base = c.take<int32_t>(b->num_seqs + 1);
+    p->block_rows = c.take<RowDesc>(nq);
+    p->token_rows = c.take<RowDesc>(nq);
+    p->mid = c.take<int32_t>(size_t(nq) * keep);
+    p->kept = c.take<int32_t>(size_t(nq) * (keep + 2));
+    const int32_t max_mid = std::max(0, (hi.max_k + B - 1) / B - 2);   // as hisa_index scores them
+    const int64_t ld_blk = score_ld(max_mid), ld_tok = score_ld((keep + 2) * B);
+    const size_t s_blk = size_t(chunk_rows(nq, ld_blk)) * ld_blk;
+    const size_t s_tok = size_t(chunk_rows(nq, ld_tok)) * ld_tok;
+    p->S = c.take<float>(std::max(s_blk, s_tok));
+    return c.off;
+}
+
+dsa_status clear_status(void* ws, cudaStream_t st)
+{
+    return cudaMemsetAsync(ws, 0, kStatusBytes, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+}  // namespace
+
+// =====================================================================
+extern "C" {
+
+const char* dsa_status_string(dsa_status s)
+{
+    switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case DSA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_DEVICE_CHECK: return "a kernel recorded a device-side error";
+    }
+    return "unknown status";
+}
+
+int32_t dsa_version(void) { return 100; }
+
+// ------------------------------------------------------------ dense scores
+size_t dsa_index_scores_workspace(const dsa_batch* b)
+{
+    HostInfo hi;
+    if (check_batch(b, &hi) != DSA_OK) return 0;
+    DensePlan p;
+    return dense_plan(nullptr, b, hi, true, &p);
+}
+
+dsa_status dsa_index_scores(const dsa_batch* b, const void* Q, const void* K, const float* W, float* S,
+                            int64_t ld_s, void* ws, size_t ws_bytes, void* stream)
+{
+    HostInfo hi;
+    dsa_status s = check_batch(b, &hi);
+    if (s != DSA_OK) return s;
+    if ((s = check_tensors(b, Q, K, W)) != DSA_OK) return s;
+    if (b->num_queries > 0 && (!S || ld_s < hi.max_k || ld_s > INT32_MAX)) return DSA_ERR_INVALID_ARG;
+    DensePlan p;
+    if ((s = check_ws(ws, ws_bytes, dense_plan(nullptr, b, hi, true, &p))) != DSA_OK) return s;
+    dense_plan(static_cast<char*>(ws), b, hi, true, &p);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = clear_status(ws, st)) != DSA_OK) return s;
+    if (b->num_queries == 0) return DSA_OK;
+    DSA_LAUNCH(kProfSetup, st, dense_rows_kernel<<<(b->num_queries + 255) / 256, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos,
+                                                                    b->num_seqs, b->num_queries, p.rows));
+    if ((s = launched()) != DSA_OK) return s;
+    return launch_score<__nv_bfloat16>(p.rows, b->num_queries, hi.max_k, identity_map(), Q, W, b->num_heads,
+                                       b->head_dim, static_cast<const __nv_bfloat16*>(K), b->k_offsets, S, ld_s,
+                                       (int32_t)ld_s, st);
+}
+
+// ------------------------------------------------------------- dense top-k
+size_t dsa_index_topk_workspace(const dsa_batch* b, int32_t k)
+{
+    HostInfo hi;
+    if (check_batch(b, &hi) != DSA_OK || k < 1 || k > kMaxK) return 0;
+    DensePlan p;
+    return dense_plan(nullptr, b, hi, false, &p);
+}
+
+dsa_status dsa_index_topk(const dsa_batch* b, const void* Q, const void* K, const float* W, int32_t k,
+                          int32_t* idx, float* scores, void* ws, size_t ws_bytes, void* stream)
+{
+    HostInfo hi;
+    dsa_status s = check_batch(b, &hi);
+    if (s != DSA_OK) return s;
+    if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
+    if ((s = check_tensors(b, Q, K, W)) != DSA_OK) return s;
+    if (b->num_queries > 0 && !idx) return DSA_ERR_INVALID_ARG;
+    DensePlan p;
+    if ((s = check_ws(ws, ws_bytes, dense_plan(nullptr, b, hi, false, &p))) != DSA_OK) return s;
+    dense_plan(static_cast<char*>(ws), b, hi, false, &p);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = clear_status(ws, st)) != DSA_OK) return s;
+    if (b->num_queries == 0) return DSA_OK;
+    DSA_LAUNCH(kProfSetup, st, dense_rows_kernel<<<(b->num_queries + 255) / 256, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos,
+                                                                    b->num_seqs, b->num_queries, p.rows));
+    if ((s = launched()) != DSA_OK) return s;
+    return score_and_select<__nv_bfloat16>(p.rows, b->num_queries, hi.max_k, identity_map(), Q, W, b->num_heads,
+                                           b->head_dim, static_cast<const __nv_bfloat16*>(K), b->k_offsets, p.S,
+                                           k, idx, k, scores, st);
+}
+
+// ------------------------------------------------------------------ PIVOT
+int32_t pivot_num_groups(const dsa_batch* b, int32_t group)
+{
+    HostInfo hi;
+    if (check_batch(b, &hi) != DSA_OK || group < 1) return -1;
+    return count_groups(b, group);
+}
+
+static bool pivot_args_ok(int32_t k, int32_t G, int32_t C, int32_t mode)
+{
+    return k >= 1 && k <= kMaxK && G >= 1 && G <= 64 && C >= k && C <= kMaxCand && (mode == 0 || mode == 1);
+}
+
+size_t pivot_group_index_workspace(const dsa_batch* b, int32_t k, int32_t G, int32_t C, int32_t mode)
+{
+    HostInfo hi;
+    if (check_batch(b, &hi) != DSA_OK || !pivot_args_ok(k, G, C, mode)) return 0;
+    PivotPlan p;
+    return pivot_plan(nullptr, b, hi, G, C, &p);
+}
+
+dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, const float* W, int32_t k,
+                             int32_t G, int32_t C, int32_t mode, int32_t* idx, int32_t* cand_out, void* ws,
+                             size_t ws_bytes, void* stream)
+{
+    HostInfo hi;
+    dsa_status s = check_batch(b, &hi);
+    if (s != DSA_OK) return s;
+    if (!pivot_args_ok(k, G, C, mode)) return DSA_ERR_UNSUPPORTED;
+    if ((s = check_tensors(b, Q, K, W)) != DSA_OK) return s;
+    if (b->num_queries > 0 && !idx) return DSA_ERR_INVALID_ARG;
+    PivotPlan p;
+    if ((s = check_ws(ws, ws_bytes, pivot_plan(nullptr, b, hi, G, C, &p))) != DSA_OK) return s;
+    pivot_plan(static_cast<char*>(ws), b, hi, G, C, &p);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = clear_status(ws, st)) != DSA_OK) return s;
+    const int32_t ng = count_groups(b, G);
+    if (ng == 0) return DSA_OK;
+    const int H = b->num_heads, D = b->head_dim;
+    int32_t* cand = cand_out ? cand_out : p.cand;
+
+    DSA_LAUNCH(kProfSetup, st, pivot_groups_kernel<<<1, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos, b->num_seqs, G, ng, p.group_base,
+                                           p.groups, p.proxy_rows));
+    if ((s = launched()) != DSA_OK) return s;
+    DSA_LAUNCH(kProfProxy, st, pivot_proxy_kernel<<<ng, 256, 0, st>>>(p.groups, static_cast<const __nv_bfloat16*>(Q), W, H, D, p.Qp, p.Wp));
+    if ((s = launched()) != DSA_OK) return s;
+    // Shared scan: each proxy against its prefix, top-C kept with their proxy scores.
+    s = score_and_select<__nv_bfloat16>(p.proxy_rows, ng, hi.max_k, identity_map(), p.Qp, p.Wp, H, D,
+                                        static_cast<const __nv_bfloat16*>(K), b->k_offsets, p.S, C, cand, C,
+                                        p.cand_score, st);
+    if (s != DSA_OK) return s;
+    DSA_LAUNCH(kProfSetup, st, pivot_query_rows_kernel<<<(b->num_queries + 255) / 256, 256, 0, st>>>(
+        b->q_offsets, b->k_offsets, b->q_pos, b->num_seqs, b->num_queries, G, p.group_base, cand, C, p.query_rows));
+    if ((s = launched()) != DSA_OK) return s;
+    ColMap m{};
+    m.kind = kMapList;
+    m.list = cand;
+    m.list_ld = C;
+    if (mode == 0) {
+        // Reuse: rank the group's candidates by their proxy scores inside each query's prefix.
+        return launch_select(p.query_rows, b->num_queries, C, k, m, p.cand_score, C, true, idx, k, nullptr, 0, st);
+    }
+    // Refine: each query scores its eligible candidates with its own indexer.
+    return score_and_select<__nv_bfloat16>(p.query_rows, b->num_queries, C, m, Q, W, H, D,
+                                           static_cast<const __nv_bfloat16*>(K), b->k_offsets, p.S, k, idx, k,
+                                           nullptr, st);
+}
+
+// ------------------------------------------------------------------- HISA
+static bool hisa_args_ok(int32_t k, int32_t B, int32_t keep)
+{
+    return k >= 1 && k <= kMaxK && (B == 64 || B == 128 || B == 256) && keep >= 1 && keep <= 256;
+}
+
+int64_t hisa_num_blocks(const dsa_batch* b, int32_t B)
+{
+    HostInfo hi;
+    if (check_batch(b, &hi) != DSA_OK || B < 1) return -1;
+    int64_t n = 0;
+    for (int i = 0; i < b->num_seqs; ++i) n += (b->k_offsets_host[i + 1] - b->k_offsets_host[i] + B - 1) / B;
+    return n;
+}
+
+dsa_status hisa_pool_keys(const dsa_batch* b, const void* K, int32_t B, float* pooled, void* stream)
+{
+    HostInfo hi;
+    dsa_status s = check_batch(b, &hi);
+    if (s != DSA_OK) return s;
+    if (!(B == 64 || B == 128 || B == 256)) return DSA_ERR_UNSUPPORTED;
+    const int64_t nb = hisa_num_blocks(b, B);
+    if (nb == 0) return DSA_OK;
+    if (!K || !pooled || (reinterpret_cast<uintptr_t>(K) & 15) || (reinterpret_cast<uintptr_t>(pooled) & 15))
+        return DSA_ERR_INVALID_ARG;
+    if (nb > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DSA_LAUNCH(kProfPool, st, hisa_pool_kernel<<<(unsigned)nb, b->head_dim, 0, st>>>(static_cast<const __nv_bfloat16*>(K), b->k_offsets,
+                                                          b->num_seqs, B, b->head_dim, pooled));
+    return launched();
+}
+
+size_t hisa_index_workspace(const dsa_batch* b, int32_t k, int32_t B, int32_t keep)
+{
+    HostInfo hi;
+    if (check_batch(b, &hi) != DSA_OK || !hisa_args_ok(k, B, keep)) return 0;
+    HisaPlan p;
+    return hisa_plan(nullptr, b, hi, B, keep, &p);
+}
+
+dsa_status hisa_index(const dsa_batch* b, const void* Q, const void* K, const float* W, const float* pooled,
+                      int32_t k, int32_t B, int32_t keep, int32_t* idx, int32_t* kept_out, void* ws, size_t ws_bytes,
+                      void* stream)
+{
+    HostInfo hi;
+    dsa_status s = check_batch(b, &hi);
+    if (s != DSA_OK) return s;
+    if (!hisa_args_ok(k, B, keep)) return DSA_ERR_UNSUPPORTED;
+    if ((s = check_tensors(b, Q, K, W)) != DSA_OK) return s;
+    if (b->num_queries > 0 && (!idx || !pooled)) return DSA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(pooled) & 15) return DSA_ERR_INVALID_ARG;
+    HisaPlan p;
+    if ((s = check_ws(ws, ws_bytes, hisa_plan(nullptr, b, hi, B, keep, &p))) != DSA_OK) return s;
+    hisa_plan(static_cast<char*>(ws), b, hi, B, keep, &p);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = clear_status(ws, st)) != DSA_OK) return s;
+    const int32_t nq = b->num_queries;
+    if (nq == 0) return DSA_OK;
+    const int H = b->num_heads, D = b->head_dim;
+    int32_t* kept = kept_out ? kept_out : p.kept;
+    const unsigned g = (nq + 255) / 256;
+
+    DSA_LAUNCH(kProfSetup, st, hisa_block_base_kernel<<<1, 32, 0, st>>>(b->k_offsets, b->num_seqs, B, p.block_base));
+    DSA_LAUNCH(kProfSetup, st, hisa_block_rows_kernel<<<g, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos, b->num_seqs, nq, B,
+                                              p.block_rows));
+    if ((s = launched()) != DSA_OK) return s;
+    // Coarse stage: middle blocks scored on their pooled keys, top `keep` kept.
+    const int32_t max_mid = std::max(0, (hi.max_k + B - 1) / B - 2);
+    s = score_and_select<float>(p.block_rows, nq, max_mid, identity_map(1), Q, W, H, D, pooled, p.block_base, p.S,
+                                keep, p.mid, keep, nullptr, st);
+    if (s != DSA_OK) return s;
+    DSA_LAUNCH(kProfSetup, st, hisa_kept_kernel<<<g, 256, 0, st>>>(p.block_rows, p.mid, keep, b->q_pos, b->k_offsets, nq, B, kept,
+                                        p.token_rows));
+    if ((s = launched()) != DSA_OK) return s;
+    // Fine stage: the indexer over the tokens of the kept blocks.
+    ColMap m{};
+    m.kind = kMapBlocks;
+    m.block = B;
+    m.list = kept;
+    m.list_ld = keep + 2;
+    return score_and_select<__nv_bfloat16>(p.token_rows, nq, (keep + 2) * B, m, Q, W, H, D,
+                                           static_cast<const __nv_bfloat16*>(K), b->k_offsets, p.S, k, idx, k,
+                                           nullptr, st);
+}
+
+// ---------------------------------------------------------------- profiling
+void dsa_profile_enable(int32_t on)
+{
+    g_prof_on.store(on != 0);
+}
+
+uint64_t dsa_launch_count(void)
+{
+    return g_launches.load();
+}
+
+const char* dsa_profile_kind_name(int32_t kind)
+{
+    return (kind >= 0 && kind < kProfKinds) ? kProfNames[kind] : nullptr;
+}
+
+int32_t dsa_profile_read(float* ms, int32_t* launches, int32_t cap)
+{
+    std::vector<ProfRec> recs;
+    {
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        recs.swap(g_prof);
+    }
+    for (int32_t k = 0; k < cap && k < kProfKinds; ++k) {
+        if (ms) ms[k] = 0.f;
+        if (launches) launches[k] = 0;
+    }
+    int32_t status = kProfKinds;
+    for (const ProfRec& r : recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+            status = -1;
+        if (r.kind < cap) {
+            if (ms) ms[r.kind] += t;
+            if (launches) launches[r.kind] += 1;
+        }
+        cudaEventDestroy(r.start);
+        cudaEventDestroy(r.stop);
+    }
+    return status;
+}
+
+// ------------------------------------------------------------ device check
+dsa_status dsa_device_check(void* ws, void* stream, uint32_t* detail)
+{
+    if (!ws) return DSA_ERR_INVALID_ARG;
+    uint32_t h[2] = {0, 0};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(h, ws, sizeof h, cudaMemcpyDeviceToHost, st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (h[0] == 0) return DSA_OK;
+    if (detail) *detail = h[0];
+    if (cudaMemsetAsync(ws, 0, 8, st) != cudaSuccess) return DSA_ERR_CUDA;
+    return DSA_ERR_DEVICE_CHECK;
+}
+
+}  // extern "C"

@@ -1,0 +1,219 @@
+// Small kernels that lay out the ranking problems of each entry point:
+// row descriptors, PIVOT's groups and proxies, HISA's pooled keys and kept
+// block lists.
+#pragma once
+
+#include "common.cuh"
+
+namespace dsa {
+
+// ------------------------------------------------------------------ dense
+// One row per query: eligible keys s <= q_pos[t] of its sequence.
+__global__ void dense_rows_kernel(const int32_t* q_off, const int32_t* k_off, const int32_t* q_pos,
+                                  int32_t n_seqs, int32_t n_q, RowDesc* rows)
+{
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n_q) return;
+    const int b = find_seq(q_off, n_seqs, t);
+    rows[t] = RowDesc{t, b, eligible_count(q_pos[t], k_off[b + 1] - k_off[b]), 0};
+}
+
+// ------------------------------------------------------------------ PIVOT
+// PIVOT ("PIVOT: Efficient Query-Group Indexing for Token-Level Sparse
+// Attention", abstract): inside each sequence, consecutive runs of G query
+// rows form a group; the group's proxy scans keys up to its last position.
+struct GroupDesc {
+    int32_t seq;
+    int32_t first;    // first query row
+    int32_t size;     // queries in the group (<= G)
+    int32_t n_scan;   // keys the proxy scans: s < n_scan
+};
+
+// Single CTA: group_base[b] = number of groups before sequence b, then one
+// GroupDesc and one proxy RowDesc per group.
+__global__ void pivot_groups_kernel(const int32_t* q_off, const int32_t* k_off, const int32_t* q_pos,
+                                    int32_t n_seqs, int32_t G, int32_t n_groups, int32_t* group_base,
+                                    GroupDesc* groups, RowDesc* proxy_rows)
+{
+    if (threadIdx.x == 0) {
+        int32_t acc = 0;
+        for (int b = 0; b < n_seqs; ++b) {
+            group_base[b] = acc;
+            acc += (q_off[b + 1] - q_off[b] + G - 1) / G;
+        }
+        group_base[n_seqs] = acc;
+    }
+    __syncthreads();
+    for (int g = threadIdx.x; g < n_groups; g += blockDim.x) {
+        const int b = find_seq(group_base, n_seqs, g);
+        const int first = q_off[b] + (g - group_base[b]) * G;
+        const int size = min(G, q_off[b + 1] - first);
+        int32_t p_last = -1;
+        for (int j = 0; j < size; ++j) p_last = max(p_last, q_pos[first + j]);
+        const int n_scan = eligible_count(p_last, k_off[b + 1] - k_off[b]);
+        groups[g] = GroupDesc{b, first, size, n_scan};
+        proxy_rows[g] = RowDesc{g, b, n_scan, g};
+    }
+}
+
+// Nearest bf16 of a double, ties to even, from the format: 1 sign bit, 8
+// exponent bits, 7 stored significand bits.  The double's 52-bit significand
+// is cut after its top 7 bits and rounded on the 45 bits cut off; values
+// below the smallest normal bf16 (2^-126) are rounded on the subnormal grid
+// 2^-133.  Values stay far below the bf16 overflow threshold.
+__device__ __forceinline__ uint16_t bf16_bits_rne(double x)
+{
+    const uint64_t u = (uint64_t)__double_as_longlong(x);
+    const uint32_t sign = (uint32_t)(u >> 63) << 15;
+    const int e = (int)((u >> 52) & 0x7ff) - 1023;
+    if (x == 0.0) return (uint16_t)sign;
+    if (e < -126) {
+        const double m = fabs(x) * 0x1p133;           // exact power-of-two scaling
+        const double r = rint(m);                       // ties to even
+        return (uint16_t)(sign | (uint32_t)r);          // r == 128 encodes 2^-126
+    }
+    uint64_t mant = u & ((1ull << 52) - 1);
+    uint64_t keep = mant >> 45;
+    const uint64_t rest = mant & ((1ull << 45) - 1);
+    const uint64_t half = 1ull << 44;
+    uint32_t ex = (uint32_t)(e + 127);
+    if (rest > half || (rest == half && (keep & 1))) {
+        if (++keep == 128) { keep = 0; ++ex; }
+    }
+    return (uint16_t)(sign | (ex << 7) | (uint32_t)keep);
+}
+
+// One CTA per group: proxy q = bf16(mean of q) with the mean in double,
+// proxy w = mean of w (double, stored fp32).
+__global__ void pivot_proxy_kernel(const GroupDesc* groups, const __nv_bfloat16* Q, const float* W,
+                                   int32_t H, int32_t D, __nv_bfloat16* Qp, float* Wp)
+{
+    const GroupDesc g = groups[blockIdx.x];
+    const int HD = H * D;
+    const uint16_t* q = reinterpret_cast<const uint16_t*>(Q);
+    uint16_t* qp = reinterpret_cast<uint16_t*>(Qp) + (int64_t)blockIdx.x * HD;
+    for (int e = threadIdx.x; e < HD; e += blockDim.x) {
+        double s = 0.0;
+        for (int j = 0; j < g.size; ++j)
+            s += (double)__uint_as_float((uint32_t)q[(int64_t)(g.first + j) * HD + e] << 16);
+        qp[e] = bf16_bits_rne(s / g.size);
+    }
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+        double s = 0.0;
+        for (int j = 0; j < g.size; ++j) s += (double)W[(int64_t)(g.first + j) * H + h];
+        Wp[(int64_t)blockIdx.x * H + h] = (float)(s / g.size);
+    }
+}
+
+// One row per query for Reuse / Refine: the group's candidates (ascending,
+// -1 padded) that lie inside the query's own prefix form a prefix of the
+// candidate list; RowDesc.list = group.
+__global__ void pivot_query_rows_kernel(const int32_t* q_off, const int32_t* k_off, const int32_t* q_pos,
+                                        int32_t n_seqs, int32_t n_q, int32_t G, const int32_t* group_base,
+                                        const int32_t* cand, int32_t C, RowDesc* rows)
+{
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n_q) return;
+    const int b = find_seq(q_off, n_seqs, t);
+    const int g = group_base[b] + (t - q_off[b]) / G;
+    const int lim = eligible_count(q_pos[t], k_off[b + 1] - k_off[b]);   // keys s < lim
+    const int32_t* c = cand + (int64_t)g * C;
+    int lo = 0, hi = C;   // first position whose candidate is >= lim or -1
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        const int32_t s = c[mid];
+        if (s >= 0 && s < lim) lo = mid + 1; else hi = mid;
+    }
+    rows[t] = RowDesc{t, b, lo, g};
+}
+
+// ------------------------------------------------------------------- HISA
+// HISA ("HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse
+// Attention", abstract): pooled block keys, block filter, token refinement.
+
+// Single CTA: block_base[b] = pooled blocks before sequence b.
+__global__ void hisa_block_base_kernel(const int32_t* k_off, int32_t n_seqs, int32_t B, int32_t* block_base)
+{
+    if (threadIdx.x == 0 && blockIdx.x == 0) {
+        int32_t acc = 0;
+        for (int b = 0; b < n_seqs; ++b) {
+            block_base[b] = acc;
+            acc += (k_off[b + 1] - k_off[b] + B - 1) / B;
+        }
+        block_base[n_seqs] = acc;
+    }
+}
+
+// Pooled key of block j: mean of its keys (fp32 sum in token order).  One
+// CTA of D threads per block; thread i owns dimension i (coalesced rows).
+// The owning sequence is found by walking the key offsets (few sequences).
+__global__ void hisa_pool_kernel(const __nv_bfloat16* K, const int32_t* k_off, int32_t n_seqs, int32_t B,
+                                 int32_t D, float* pooled)
+{
+    __shared__ int32_t s_seq, s_first;
+    const int j = blockIdx.x;
+    if (threadIdx.x == 0) {
+        int32_t acc = 0, b = 0;
+        for (; b < n_seqs; ++b) {
+            const int32_t nb = (k_off[b + 1] - k_off[b] + B - 1) / B;
+            if (j < acc + nb) break;
+            acc += nb;
+        }
+        s_seq = b;
+        s_first = acc;
+    }
+    __syncthreads();
+    const int b = s_seq;
+    const int s0 = (j - s_first) * B;
+    const int L = k_off[b + 1] - k_off[b];
+    const int s1 = min(s0 + B, L);
+    const uint16_t* k = reinterpret_cast<const uint16_t*>(K) + (int64_t)k_off[b] * D;
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+        float s = 0.f;
+        for (int t = s0; t < s1; ++t) s += __uint_as_float((uint32_t)k[(int64_t)t * D + i] << 16);
+        pooled[(int64_t)j * D + i] = s / (float)(s1 - s0);
+    }
+}
+
+// Block-scoring rows: the middle blocks 1 .. last-1 of query t (column c is
+// block c + 1).
+__global__ void hisa_block_rows_kernel(const int32_t* q_off, const int32_t* k_off, const int32_t* q_pos,
+                                       int32_t n_seqs, int32_t n_q, int32_t B, RowDesc* rows)
+{
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n_q) return;
+    const int b = find_seq(q_off, n_seqs, t);
+    const int n = eligible_count(q_pos[t], k_off[b + 1] - k_off[b]);
+    const int last = n > 0 ? (n - 1) / B : 0;
+    rows[t] = RowDesc{t, b, last > 1 ? last - 1 : 0, t};
+}
+
+// Kept blocks of query t: block 0, the selected middle blocks (ascending,
+// -1 padded), and the query's own block; then the token row over them.
+__global__ void hisa_kept_kernel(const RowDesc* block_rows, const int32_t* mid, int32_t keep,
+                                 const int32_t* q_pos, const int32_t* k_off, int32_t n_q, int32_t B,
+                                 int32_t* kept, RowDesc* token_rows)
+{
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n_q) return;
+    const RowDesc br = block_rows[t];
+    const int n = eligible_count(q_pos[t], k_off[br.seq + 1] - k_off[br.seq]);
+    int32_t* out = kept + (int64_t)t * (keep + 2);
+    int m = 0;
+    int ncols = 0;
+    if (n > 0) {
+        const int last = (n - 1) / B;
+        out[m++] = 0;
+        for (int j = 0; j < keep; ++j) {
+            const int32_t v = mid[(int64_t)t * keep + j];
+            if (v < 0) break;
+            out[m++] = v;
+        }
+        if (last > 0) out[m++] = last;
+        ncols = (m - 1) * B + (n - last * B);
+    }
+    for (int j = m; j < keep + 2; ++j) out[j] = -1;
+    token_rows[t] = RowDesc{t, br.seq, ncols, t};
+}
+
+}  // namespace dsa

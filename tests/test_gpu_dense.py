@@ -1,0 +1,119 @@
+"""GPU parity of the dense indexer (scores and top-k) against the oracle.
+
+Integer-valued inputs: exact (fp32 scores bit-equal to the fp64 oracle,
+index sets equal, ties to the lower index).  bf16 inputs: the tolerance rule
+of tests/parity.py (relative 2e-3 of max(|k-th score|, row RMS)).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import check_exact_sets, check_scores_close, check_tolerance_rows
+from gpu_util import Dev, ascending_packed
+
+pytestmark = pytest.mark.gpu
+
+
+def exact_topk(b, k):
+    d = Dev(b)
+    idx, sc = d.topk(k, want_scores=True)
+    ref = oracle.dense(b, k=k, want_all=True)
+    ascending_packed(idx)
+    check_exact_sets(idx, ref["idx"])
+    # returned scores: exactly the oracle's score of each returned index
+    for t in range(b.n_q):
+        v = idx[t] >= 0
+        assert np.array_equal(sc[t][v].astype(np.float64), ref["all"][t][idx[t][v]]), t
+        assert np.all(np.isnan(sc[t][~v]))
+    return d, ref
+
+
+def test_tiny_integer_prefill_exact():
+    b = workloads.tiny_integer(seed=0, T=512, H=4, d=32, k=64)
+    d, ref = exact_topk(b, 64)
+    S = d.scores()
+    assert np.array_equal(S.astype(np.float64), ref["all"])
+
+
+def test_signed_weights_exact():
+    exact_topk(workloads.tiny_integer(seed=1, T=300, H=4, d=32, k=40, signed_w=True), 40)
+
+
+@pytest.mark.parametrize("H,dim", [(1, 32), (8, 64), (16, 128), (64, 32), (2, 128)])
+def test_head_shapes_exact(H, dim):
+    exact_topk(workloads.tiny_integer(seed=H + dim, T=260, H=H, d=dim, k=33), 33)
+
+
+@pytest.mark.parametrize("seed,q_lens,k_lens,mode", [
+    (10, [5, 1, 64], [300, 17, 129], "random"),
+    (11, [200, 3], [200, 1000], "suffix"),
+    (12, [1, 1, 1, 1], [1, 2, 130, 257], "suffix"),
+    (13, [0, 40, 0], [10, 40, 5], "random"),
+])
+def test_ragged_batches_exact(seed, q_lens, k_lens, mode):
+    exact_topk(workloads.ragged(seed, q_lens, k_lens, H=4, d=32, k=24, integer=True, pos_mode=mode), 24)
+
+
+def test_k_larger_than_every_row():
+    b = workloads.tiny_integer(seed=2, T=200, H=4, d=32, k=300)
+    exact_topk(b, 300)
+
+
+def test_all_equal_scores_take_lowest_indices():
+    b = workloads.tiny_integer(seed=3, T=400, H=4, d=32, k=50)
+    b.K = torch.ones_like(b.K)
+    b.Q = torch.ones_like(b.Q)
+    idx = Dev(b).topk(50)
+    for t in range(b.n_q):
+        n = min(50, t + 1)
+        assert idx[t].tolist() == list(range(n)) + [-1] * (50 - n)
+
+
+def test_empty_query_batch():
+    b = workloads.ragged(4, [0], [10], H=4, d=32, k=8)
+    d = Dev(b)
+    assert d.topk(8).shape == (0, 8)
+
+
+def test_bf16_prefill_tolerance():
+    b = workloads.dense_prefill(seed=21, T=700, H=64, d=128, k=100)
+    d = Dev(b)
+    idx = d.topk(100)
+    ascending_packed(idx)
+    ref = oracle.dense(b, k=100, want_all=True)
+    check_tolerance_rows(idx, ref["idx"], ref["all"])
+    check_scores_close(d.scores(), ref["all"])
+
+
+def test_bf16_decode_tolerance():
+    b = workloads.dense_decode(seed=22, B=3, L=3000, n_mtp=2, H=64, d=128, k=256)
+    d = Dev(b)
+    idx = d.topk(256)
+    ascending_packed(idx)
+    ref = oracle.dense(b, k=256, want_all=True)
+    check_tolerance_rows(idx, ref["idx"], ref["all"])
+
+
+def test_full_size_decode_32k():
+    """Dense decode, 16 sequences x 32K keys, 2 MTP queries each, H=64, d=128, k=2048: every row."""
+    b = workloads.dense_decode(seed=1)
+    idx = Dev(b).topk(2048)
+    ascending_packed(idx)
+    ref = oracle.dense(b, k=2048, want_all=True)
+    check_tolerance_rows(idx, ref["idx"], ref["all"])
+
+
+def test_full_size_prefill_32k_sampled_rows():
+    """Dense prefill T = L = 32K, H=64, d=128, k=2048: the whole batch on the GPU, sampled rows checked."""
+    b = workloads.dense_prefill(seed=2)
+    idx = Dev(b).topk(2048)
+    rows = workloads.stratified_rows(b.n_q, n_sample=40, head=8, tail=8)
+    ref = oracle.dense(b, rows=rows, k=2048, want_all=True)
+    ascending_packed(idx[rows])
+    check_tolerance_rows(idx[rows], ref["idx"], ref["all"])
+    # every row holds min(k, t+1) indices, all causal
+    counts = (idx >= 0).sum(1)
+    assert np.array_equal(counts, np.minimum(np.arange(b.n_q) + 1, 2048))
+    assert np.all(idx.max(1) <= np.arange(b.n_q))

@@ -1,0 +1,160 @@
+"""GPU parity of PIVOT (Reuse / Refine) and HISA against the oracle.
+
+Both methods are two-stage.  The first stage (PIVOT candidates, HISA kept
+blocks) is compared with the oracle's under the same rule as the final
+indices; the second stage is compared with the oracle's second stage run on
+the GPU's own first-stage result (identical when the first stages agree).
+Integer-valued inputs with power-of-two group sizes keep every proxy, pooled
+key and score exact, so those cases are compared exactly.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from parity import check_exact_sets, check_tolerance_row
+from gpu_util import Dev, ascending_packed
+
+pytestmark = pytest.mark.gpu
+
+
+def group_rows(b, G):
+    """Oracle output row of each query (groups are padded to G rows)."""
+    rows = []
+    qo = b.q_offsets.tolist()
+    g0 = 0
+    for s in range(b.num_seqs):
+        nq = qo[s + 1] - qo[s]
+        for j in range(nq):
+            rows.append((g0 + j // G) * G + j % G)
+        g0 += (nq + G - 1) // G
+    return np.array(rows, dtype=np.int64)
+
+
+# ------------------------------------------------------------------ PIVOT
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("G,C,k", [(16, 256, 64), (4, 64, 64), (1, 64, 64)])
+def test_pivot_integer_exact(mode, G, C, k):
+    b = workloads.tiny_integer(seed=5, T=512, H=4, d=32, k=k)
+    idx, cand = Dev(b).pivot(k, G, C, mode)
+    ref = oracle.pivot(b, G, C, k)
+    ascending_packed(cand)
+    check_exact_sets(cand, ref["cand"], "cand")
+    r = group_rows(b, G)
+    check_exact_sets(idx, (ref["reuse_idx"] if mode == 0 else ref["refine_idx"])[r], "idx")
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_pivot_ragged_integer_exact(mode):
+    b = workloads.ragged(7, [37, 64, 5], [37, 200, 90], H=4, d=32, k=16, integer=True)
+    G, C, k = 8, 40, 16
+    idx, cand = Dev(b).pivot(k, G, C, mode)
+    ref = oracle.pivot(b, G, C, k)
+    check_exact_sets(cand, ref["cand"], "cand")
+    r = group_rows(b, G)
+    check_exact_sets(idx, (ref["reuse_idx"] if mode == 0 else ref["refine_idx"])[r], "idx")
+
+
+def check_pivot_bf16(b, G, C, k, mode):
+    idx, cand = Dev(b).pivot(k, G, C, mode)
+    own = oracle.pivot(b, G, C, k)                      # the oracle's own two stages
+    ext = oracle.pivot(b, G, C, k, ext_cand=cand)       # its second stage on the GPU's candidates
+    ascending_packed(cand)
+    # stage 1: candidate sets under the rule, scored by the oracle's proxy
+    for g in range(cand.shape[0]):
+        sc = {}
+        for src in (own, ext):
+            v = src["cand"][g] >= 0
+            sc.update(zip(src["cand"][g][v].tolist(), src["cand_score"][g][v].tolist()))
+        rms = float(np.sqrt(np.mean(own["cand_score"][g][own["cand"][g] >= 0] ** 2)))
+        msg = check_tolerance_row(cand[g], own["cand"][g], lambda ix: np.array([sc[x] for x in ix]), rms)
+        assert msg is None, f"group {g} candidates: {msg}"
+    # stage 2: each query against the oracle's second stage on the same candidates
+    rows = group_rows(b, G)
+    for t in range(b.n_q):
+        g = rows[t] // G
+        v = (ext["cand"][g] >= 0) & (ext["cand"][g] <= int(b.q_pos[t]))
+        elig = ext["cand"][g][v]
+        if mode == 0:
+            prox = dict(zip(elig.tolist(), ext["cand_score"][g][v].tolist()))
+            score_of = lambda ix, d=prox: np.array([d[x] for x in ix])
+            ref_row = ext["reuse_idx"][rows[t]]
+        else:
+            own_sc = dict(zip(elig.tolist(), oracle.pair_scores(b, [t] * elig.size, elig).tolist()))
+            score_of = lambda ix, d=own_sc: np.array([d[x] for x in ix])
+            ref_row = ext["refine_idx"][rows[t]]
+        fin = score_of(elig) if elig.size else np.zeros(1)
+        rms = float(np.sqrt(np.mean(fin ** 2)))
+        msg = check_tolerance_row(idx[t], ref_row, score_of, rms)
+        assert msg is None, f"query {t}: {msg}"
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_pivot_bf16_small(mode):
+    b = workloads.dense_prefill(seed=31, T=600, H=64, d=128, k=64)
+    check_pivot_bf16(b, G=16, C=256, k=64, mode=mode)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_pivot_decode_groups_are_mtp_steps(mode):
+    """Decode: a group is the MTP queries of one step (group size = queries per sequence)."""
+    b = workloads.dense_decode(seed=32, B=4, L=2000, n_mtp=2, H=64, d=128, k=128)
+    check_pivot_bf16(b, G=2, C=512, k=128, mode=mode)
+
+
+# ------------------------------------------------------------------- HISA
+
+def test_hisa_pool_integer_exact():
+    b = workloads.ragged(8, [1, 1], [1000, 300], H=4, d=32, k=8, integer=True)
+    _, _, pooled = Dev(b).hisa(8, 64, 4)
+    assert np.array_equal(pooled.astype(np.float64), oracle.hisa_pool(b, 64))
+
+
+@pytest.mark.parametrize("B,keep", [(64, 3), (128, 1), (64, 40)])
+def test_hisa_integer_exact(B, keep):
+    b = workloads.ragged(9, [3, 2, 4], [1500, 700, 129], H=4, d=32, k=100, integer=True, pos_mode="random")
+    idx, kept, _ = Dev(b).hisa(100, B, keep)
+    ref = oracle.hisa(b, B, keep, 100)
+    check_exact_sets(kept, ref["kept"], "kept")
+    check_exact_sets(idx, ref["idx"], "idx")
+
+
+def check_hisa_bf16(b, k, B, keep):
+    idx, kept, pooled = Dev(b).hisa(k, B, keep)
+    ascending_packed(kept)
+    own = oracle.hisa(b, B, keep, k)
+    for t in range(b.n_q):
+        bs = own["block_scores"][t]
+        mid = np.nonzero(~np.isnan(bs))[0]
+        rms = float(np.sqrt(np.mean(bs[mid] ** 2))) if mid.size else 0.0
+        strip = lambda r: r[(r >= 0)][1:-1] if (r >= 0).sum() > 1 else r[:0]
+        gk, ok = kept[t], own["kept"][t]
+        if mid.size:
+            g_mid = np.concatenate([strip(gk), -np.ones(keep + 2, np.int32)])[:keep]
+            o_mid = np.concatenate([strip(ok), -np.ones(keep + 2, np.int32)])[:keep]
+            msg = check_tolerance_row(g_mid, o_mid, lambda ix: bs[ix], rms)
+            assert msg is None, f"row {t} kept blocks: {msg}"
+    ext = oracle.hisa(b, B, keep, k, ext_kept=kept)
+    for t in range(b.n_q):
+        cols = []
+        p = int(b.q_pos[t])
+        for blk in kept[t][kept[t] >= 0]:
+            cols.extend(range(blk * B, min(blk * B + B, p + 1)))
+        sc = oracle.pair_scores(b, [t] * len(cols), cols)
+        d = dict(zip(cols, sc))
+        rms = float(np.sqrt(np.mean(sc ** 2))) if len(cols) else 0.0
+        msg = check_tolerance_row(idx[t], ext["idx"][t], lambda ix: np.array([d[x] for x in ix]), rms)
+        assert msg is None, f"row {t}: {msg}"
+
+
+def test_hisa_bf16_needles():
+    b = workloads.hisa_decode(seed=41, B=2, L=40000, n_mtp=2, H=64, d=128, k=512, block=128, keep=16,
+                              n_needles=6)
+    check_hisa_bf16(b, 512, 128, 16)
+
+
+def test_full_size_hisa_256k():
+    """HISA decode at 256K: 4 sequences, 2 queries, H=64, d=128, k=2048, block 128, keep 64 (+2)."""
+    b = workloads.hisa_decode(seed=4)
+    check_hisa_bf16(b, 2048, 128, 64)
