@@ -106,9 +106,14 @@ def test_pivot_decode_groups_are_mtp_steps(mode):
 # ------------------------------------------------------------------- HISA
 
 def test_hisa_pool_integer_exact():
+    """Integer keys: the block sums are exact in fp32, so each pooled key is the exact mean rounded once
+    to fp32 (full blocks of 64 keys are exact; the partial last blocks hold 40 and 44 keys)."""
     b = workloads.ragged(8, [1, 1], [1000, 300], H=4, d=32, k=8, integer=True)
     _, _, pooled = Dev(b).hisa(8, 64, 4)
-    assert np.array_equal(pooled.astype(np.float64), oracle.hisa_pool(b, 64))
+    ref = oracle.hisa_pool(b, 64)
+    assert np.array_equal(pooled, ref.astype(np.float32))
+    full = [j for j in range(ref.shape[0]) if j not in (15, 15 + 5)]
+    assert np.array_equal(pooled[full].astype(np.float64), ref[full])
 
 
 @pytest.mark.parametrize("B,keep", [(64, 3), (128, 1), (64, 40)])
