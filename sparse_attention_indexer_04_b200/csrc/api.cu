@@ -12,6 +12,7 @@
 #include "../../include/dsa_index.h"
 #include "common.cuh"
 #include "score_simt.cuh"
+#include "score_tc.cuh"
 #include "select.cuh"
 #include "setup.cuh"
 
@@ -88,8 +89,11 @@ dsa_status launched()
 
 // ------------------------------------------------------------- profiling
 // Kernel kinds timed by the optional profiler (dsa_profile_*).
-enum ProfKind : int32_t { kProfSetup = 0, kProfScoreSimt, kProfSelect, kProfPool, kProfProxy, kProfKinds };
-const char* const kProfNames[kProfKinds] = {"setup", "score_simt", "select_topk", "hisa_pool", "pivot_proxy"};
+enum ProfKind : int32_t {
+    kProfSetup = 0, kProfScoreSimt, kProfSelect, kProfPool, kProfProxy, kProfScoreTc, kProfFill, kProfKinds
+};
+const char* const kProfNames[kProfKinds] = {"setup", "score_simt", "select_topk", "hisa_pool", "pivot_proxy",
+                                            "score_tc", "fill"};
 
 struct ProfRec {
     int32_t kind;
@@ -201,6 +205,179 @@ dsa_status score_and_select(const RowDesc* rows, int32_t n_rows, int32_t max_col
     return DSA_OK;
 }
 
+// ------------------------------------------------------ tensor-core path
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled from the driver, found through the runtime (no link against libcuda).
+EncodeTiledFn encode_tiled()
+{
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Tensor map of a row-major [rows, D] bf16 matrix, loaded in boxes of box_rows
+// rows x (64 or 128 bytes) with the matching shared-memory swizzle; rows past
+// the end read as zeros.
+bool make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int D, int box_rows)
+{
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc || rows <= 0 || rows > INT32_MAX) return false;
+    const int row_bytes = D * 2 >= 128 ? 128 : 64;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {(cuuint32_t)(row_bytes / 2), (cuuint32_t)box_rows};
+    cuuint32_t elem[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, elem,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int32_t tc_tile_rows(int H) { return 2 * (256 / H); }
+
+int32_t tc_count_tiles(const int32_t* off, int n_seqs, int64_t row_base, int64_t n_rows, int32_t TQ)
+{
+    int64_t n = 0;
+    for (int b = 0; b < n_seqs; ++b) {
+        const int64_t lo = std::max<int64_t>(off[b], row_base), hi = std::min<int64_t>(off[b + 1], row_base + n_rows);
+        if (hi > lo) n += (hi - lo + TQ - 1) / TQ;
+    }
+    return (int32_t)n;
+}
+
+// Key-range splits per tile: enough units to fill the GPU twice over when there
+// are few query tiles (decode), each split keeping >= 8 key tiles.
+int32_t tc_splits(int32_t tiles, int32_t max_cols)
+{
+    const int32_t kt = (max_cols + 127) / 128;
+    if (tiles <= 0 || tiles >= 148 || kt < 16) return 1;
+    return std::max(1, std::min((2 * 148 + tiles - 1) / tiles, kt / 8));
+}
+
+// A query-row source for the tensor-core path: rows r of the launch read
+// Q[rd.qrow] / W[rd.qrow]; seq_off are absolute row offsets per sequence.
+struct TcSource {
+    const void* Q;
+    int64_t q_rows;
+    const float* W;
+    const int32_t* seq_off;
+    const int32_t* seq_off_host;
+    int32_t n_seqs;
+};
+
+int32_t tc_unit_capacity(const TcSource& src, int32_t n_rows, int32_t chunk, int H, int32_t max_cols)
+{
+    const int32_t TQ = tc_tile_rows(H);
+    int32_t cap = 1;
+    for (int32_t r0 = 0; r0 < n_rows; r0 += chunk) {
+        const int32_t nr = std::min(chunk, n_rows - r0);
+        const int32_t t = tc_count_tiles(src.seq_off_host, src.n_seqs, r0, nr, TQ);
+        cap = std::max(cap, t * tc_splits(t, max_cols));
+    }
+    return cap;
+}
+
+template <int D, int H>
+dsa_status launch_tc_shape(const CUtensorMap& mq, const CUtensorMap& mk, const TcArgs& a, int32_t n_units,
+                           int n_acc, cudaStream_t st)
+{
+    using SH = TcShape<D, H>;
+    const int budget = 232448;
+    int stages = (budget - (int)SH::smem_bytes(n_acc, 0)) / (int)SH::KTILE;
+    stages = std::min(stages, kTcMaxStages);
+    if (stages < 2) return DSA_ERR_UNSUPPORTED;
+    TcArgs args = a;
+    args.n_stages = stages;
+    // >= 120 KB keeps one CTA per SM, so no two CTAs ever wait on each other for the 512 TMEM columns.
+    const int smem = std::max((int)SH::smem_bytes(n_acc, stages), 120 * 1024);
+    if (cudaFuncSetAttribute(score_tc_kernel<D, H>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    DSA_LAUNCH(kProfScoreTc, st, score_tc_kernel<D, H><<<n_units, kTcThreads, smem, st>>>(mq, mk, args));
+    return launched();
+}
+
+template <int D>
+dsa_status launch_tc_d(int H, const CUtensorMap& mq, const CUtensorMap& mk, const TcArgs& a, int32_t n_units,
+                       int n_acc, cudaStream_t st)
+{
+    switch (H) {
+    case 1: return launch_tc_shape<D, 1>(mq, mk, a, n_units, n_acc, st);
+    case 2: return launch_tc_shape<D, 2>(mq, mk, a, n_units, n_acc, st);
+    case 4: return launch_tc_shape<D, 4>(mq, mk, a, n_units, n_acc, st);
+    case 8: return launch_tc_shape<D, 8>(mq, mk, a, n_units, n_acc, st);
+    case 16: return launch_tc_shape<D, 16>(mq, mk, a, n_units, n_acc, st);
+    case 32: return launch_tc_shape<D, 32>(mq, mk, a, n_units, n_acc, st);
+    default: return launch_tc_shape<D, 64>(mq, mk, a, n_units, n_acc, st);
+    }
+}
+
+// Tensor-core scores of launch rows [0, n_rows) (absolute [row_base, ...)) into
+// S[r * ld + s] for eligible keys s < rows[r].ncols.
+dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const TcSource& src, int H, int D,
+                    const void* K, int64_t n_k, const int32_t* k_base, int32_t max_cols, float* S, int64_t ld,
+                    TcUnitOut* units, int32_t* tile_base, uint32_t* status, cudaStream_t st)
+{
+    if (n_rows <= 0 || max_cols <= 0 || n_k <= 0) return DSA_OK;
+    const int32_t TQ = tc_tile_rows(H);
+    const int32_t tiles = tc_count_tiles(src.seq_off_host, src.n_seqs, row_base, n_rows, TQ);
+    if (tiles == 0) return DSA_OK;
+    const int32_t splits = tc_splits(tiles, max_cols);
+    CUtensorMap mq, mk;
+    if (!make_tile_map(&mq, src.Q, src.q_rows * H, D, 256) || !make_tile_map(&mk, K, n_k, D, 128))
+        return DSA_ERR_CUDA;
+    DSA_LAUNCH(kProfSetup, st, tc_units_kernel<<<1, 256, 0, st>>>(rows, n_rows, row_base, src.seq_off, src.n_seqs,
+                                                                   TQ, splits, tile_base, units));
+    dsa_status s = launched();
+    if (s != DSA_OK) return s;
+    int32_t max_q = 0;
+    for (int b = 0; b < src.n_seqs; ++b) max_q = std::max(max_q, src.seq_off_host[b + 1] - src.seq_off_host[b]);
+    const int n_acc = std::min(max_q, TQ) > TQ / 2 ? 2 : 1;
+    TcArgs a{};
+    a.units = reinterpret_cast<const TcUnit*>(units);
+    a.rows = rows;
+    a.W = src.W;
+    a.k_base = k_base;
+    a.S = S;
+    a.ld_s = ld;
+    a.status = status;
+    switch (D) {
+    case 32: return launch_tc_d<32>(H, mq, mk, a, tiles * splits, n_acc, st);
+    case 64: return launch_tc_d<64>(H, mq, mk, a, tiles * splits, n_acc, st);
+    default: return launch_tc_d<128>(H, mq, mk, a, tiles * splits, n_acc, st);
+    }
+}
+
+// Tensor-core scoring then exact top-k, in row chunks that fit the score buffer.
+dsa_status tc_score_and_select(const RowDesc* rows, int32_t n_rows, const TcSource& src, int H, int D, const void* K,
+                               int64_t n_k, const int32_t* k_base, int32_t max_cols, float* Sbuf, TcUnitOut* units,
+                               int32_t* tile_base, uint32_t* status, int32_t k, int32_t* idx, int64_t ld_idx,
+                               float* scores, cudaStream_t st)
+{
+    const int64_t ld = score_ld(max_cols);
+    const int32_t chunk = chunk_rows(n_rows, ld);
+    const ColMap map = ColMap{kMapIdentity, 0, 0, 0, nullptr, 0};
+    for (int32_t r0 = 0; r0 < n_rows; r0 += chunk) {
+        const int32_t nr = std::min(chunk, n_rows - r0);
+        dsa_status s = tc_score(rows + r0, nr, r0, src, H, D, K, n_k, k_base, max_cols, Sbuf, ld, units, tile_base,
+                                status, st);
+        if (s != DSA_OK) return s;
+        s = launch_select(rows + r0, nr, max_cols, k, map, Sbuf, ld, false, idx + int64_t(r0) * ld_idx, ld_idx,
+                          scores ? scores + int64_t(r0) * ld_idx : nullptr, ld_idx, st);
+        if (s != DSA_OK) return s;
+    }
+    return DSA_OK;
+}
+
 ColMap identity_map(int32_t offset = 0)
 {
     ColMap m{};
@@ -214,16 +391,21 @@ ColMap identity_map(int32_t offset = 0)
 struct DensePlan {
     RowDesc* rows;
     float* S;
+    TcUnitOut* units;
+    int32_t* tile_base;
 };
 
 size_t dense_plan(char* base, const dsa_batch* b, const HostInfo& hi, bool scores_only, DensePlan* p)
 {
     Carver c{base};
-    p->rows = c.take<RowDesc>(std::max(1, b->num_queries));
-    if (!scores_only) {
-        const int64_t ld = score_ld(hi.max_k);
-        p->S = c.take<float>(size_t(chunk_rows(std::max(1, b->num_queries), ld)) * ld);
-    }
+    const int32_t nq = std::max(1, b->num_queries);
+    p->rows = c.take<RowDesc>(nq);
+    const int64_t ld = score_ld(hi.max_k);
+    const int32_t chunk = scores_only ? nq : chunk_rows(nq, ld);
+    const TcSource src{nullptr, 0, nullptr, nullptr, b->q_offsets_host, b->num_seqs};
+    p->units = c.take<TcUnitOut>(tc_unit_capacity(src, b->num_queries, chunk, b->num_heads, hi.max_k));
+    p->tile_base = c.take<int32_t>(b->num_seqs + 1);
+    if (!scores_only) p->S = c.take<float>(size_t(chunk) * ld);
     return c.off;
 }
 
@@ -237,6 +419,8 @@ struct PivotPlan {
     int32_t* cand;
     float* cand_score;
     float* S;
+    TcUnitOut* units;
+    int32_t* tile_base;
 };
 
 int32_t count_groups(const dsa_batch* b, int32_t G)
@@ -245,6 +429,15 @@ int32_t count_groups(const dsa_batch* b, int32_t G)
     for (int i = 0; i < b->num_seqs; ++i)
         n += (b->q_offsets_host[i + 1] - b->q_offsets_host[i] + G - 1) / G;
     return (int32_t)n;
+}
+
+// Host copy of the per-sequence group offsets (what pivot_groups_kernel writes on the device).
+std::vector<int32_t> group_offsets_host(const dsa_batch* b, int32_t G)
+{
+    std::vector<int32_t> off(b->num_seqs + 1, 0);
+    for (int i = 0; i < b->num_seqs; ++i)
+        off[i + 1] = off[i] + (b->q_offsets_host[i + 1] - b->q_offsets_host[i] + G - 1) / G;
+    return off;
 }
 
 size_t pivot_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t G, int32_t C, PivotPlan* p)
@@ -260,9 +453,14 @@ size_t pivot_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t G,
     p->cand = c.take<int32_t>(size_t(ng) * C);
     p->cand_score = c.take<float>(size_t(ng) * C);
     const int64_t ld_scan = score_ld(hi.max_k), ld_ref = score_ld(C);
-    const size_t s_scan = size_t(chunk_rows(ng, ld_scan)) * ld_scan;
+    const int32_t chunk_scan = chunk_rows(ng, ld_scan);
+    const size_t s_scan = size_t(chunk_scan) * ld_scan;
     const size_t s_ref = size_t(chunk_rows(std::max(1, b->num_queries), ld_ref)) * ld_ref;
     p->S = c.take<float>(std::max(s_scan, s_ref));
+    const std::vector<int32_t> goff = group_offsets_host(b, G);
+    const TcSource src{nullptr, 0, nullptr, nullptr, goff.data(), b->num_seqs};
+    p->units = c.take<TcUnitOut>(tc_unit_capacity(src, count_groups(b, G), chunk_scan, b->num_heads, hi.max_k));
+    p->tile_base = c.take<int32_t>(b->num_seqs + 1);
     return c.off;
 }
 
@@ -343,9 +541,11 @@ dsa_status dsa_index_scores(const dsa_batch* b, const void* Q, const void* K, co
     DSA_LAUNCH(kProfSetup, st, dense_rows_kernel<<<(b->num_queries + 255) / 256, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos,
                                                                     b->num_seqs, b->num_queries, p.rows));
     if ((s = launched()) != DSA_OK) return s;
-    return launch_score<__nv_bfloat16>(p.rows, b->num_queries, hi.max_k, identity_map(), Q, W, b->num_heads,
-                                       b->head_dim, static_cast<const __nv_bfloat16*>(K), b->k_offsets, S, ld_s,
-                                       (int32_t)ld_s, st);
+    DSA_LAUNCH(kProfFill, st, fill_neg_inf_kernel<<<1184, 256, 0, st>>>(S, ld_s, b->num_queries, (int32_t)ld_s));
+    if ((s = launched()) != DSA_OK) return s;
+    const TcSource src{Q, b->num_queries, W, b->q_offsets, b->q_offsets_host, b->num_seqs};
+    return tc_score(p.rows, b->num_queries, 0, src, b->num_heads, b->head_dim, K, b->num_keys, b->k_offsets, hi.max_k,
+                    S, ld_s, p.units, p.tile_base, static_cast<uint32_t*>(ws), st);
 }
 
 // ------------------------------------------------------------- dense top-k
@@ -375,9 +575,9 @@ dsa_status dsa_index_topk(const dsa_batch* b, const void* Q, const void* K, cons
     DSA_LAUNCH(kProfSetup, st, dense_rows_kernel<<<(b->num_queries + 255) / 256, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos,
                                                                     b->num_seqs, b->num_queries, p.rows));
     if ((s = launched()) != DSA_OK) return s;
-    return score_and_select<__nv_bfloat16>(p.rows, b->num_queries, hi.max_k, identity_map(), Q, W, b->num_heads,
-                                           b->head_dim, static_cast<const __nv_bfloat16*>(K), b->k_offsets, p.S,
-                                           k, idx, k, scores, st);
+    const TcSource src{Q, b->num_queries, W, b->q_offsets, b->q_offsets_host, b->num_seqs};
+    return tc_score_and_select(p.rows, b->num_queries, src, b->num_heads, b->head_dim, K, b->num_keys, b->k_offsets,
+                               hi.max_k, p.S, p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, scores, st);
 }
 
 // ------------------------------------------------------------------ PIVOT
@@ -427,9 +627,10 @@ dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, c
     DSA_LAUNCH(kProfProxy, st, pivot_proxy_kernel<<<ng, 256, 0, st>>>(p.groups, static_cast<const __nv_bfloat16*>(Q), W, H, D, p.Qp, p.Wp));
     if ((s = launched()) != DSA_OK) return s;
     // Shared scan: each proxy against its prefix, top-C kept with their proxy scores.
-    s = score_and_select<__nv_bfloat16>(p.proxy_rows, ng, hi.max_k, identity_map(), p.Qp, p.Wp, H, D,
-                                        static_cast<const __nv_bfloat16*>(K), b->k_offsets, p.S, C, cand, C,
-                                        p.cand_score, st);
+    const std::vector<int32_t> goff = group_offsets_host(b, G);
+    const TcSource src{p.Qp, ng, p.Wp, p.group_base, goff.data(), b->num_seqs};
+    s = tc_score_and_select(p.proxy_rows, ng, src, H, D, K, b->num_keys, b->k_offsets, hi.max_k, p.S, p.units,
+                            p.tile_base, static_cast<uint32_t*>(ws), C, cand, C, p.cand_score, st);
     if (s != DSA_OK) return s;
     DSA_LAUNCH(kProfSetup, st, pivot_query_rows_kernel<<<(b->num_queries + 255) / 256, 256, 0, st>>>(
         b->q_offsets, b->k_offsets, b->q_pos, b->num_seqs, b->num_queries, G, p.group_base, cand, C, p.query_rows));

@@ -1,0 +1,285 @@
+// Tensor-core (tcgen05 / TMEM) scoring of query rows against contiguous key
+// tiles: the dense contraction of the lightning indexer with its epilogue.
+//
+// Orientation.  A key tile of 128 keys is the MMA's A operand (M = 128, one
+// key per TMEM lane); the query-head pairs of up to 256 / H queries are the B
+// operand (N = queries * H <= 256); K = d.  The fp32 accumulator row of a
+// TMEM lane therefore holds q[t,h] . k[s] for one key s and every (t, h) of
+// the tile, so each epilogue thread owns one key and reduces
+// I[t,s] = sum_h w[t,h] * max(0, q[t,h] . k[s]) in registers with no
+// cross-thread traffic.
+//
+// A CTA owns one work unit: up to 2 * (256 / H) consecutive queries of one
+// sequence (two accumulators of 256 TMEM columns each, so every key tile in
+// shared memory feeds two MMAs) and a range of its key tiles.  Roles:
+//   warp 0      TMA producer: the query tile once, then a ring of key tiles
+//   warp 1      TMEM allocator and MMA issuer (one thread)
+//   warps 2..9  epilogue: TMEM -> registers, ReLU, weighted head sum, causal
+//               mask, fp32 score store
+// The two accumulators are handed back and forth between MMA and epilogue
+// with mbarriers, so the MMAs into one overlap the epilogue of the other.
+// Every wait is bounded (1 s); a wait that runs out records an error in the
+// workspace status word and the CTA drains its copies and MMAs and exits.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace dsa {
+
+constexpr int kTcThreads = 320;
+constexpr int kTcMaxStages = 8;
+constexpr uint32_t kErrSmemAlign = 3;
+
+struct TcUnit {
+    int32_t row0;    // first row of the unit in the launch's row array
+    int32_t nrows;   // consecutive queries of one sequence
+    int32_t kt0;     // key tiles [kt0, kt1) of 128 keys, sequence-local
+    int32_t kt1;
+};
+
+struct TcArgs {
+    const TcUnit* units;
+    const RowDesc* rows;
+    const float* W;          // row rd.qrow: [H]
+    const int32_t* k_base;   // key row of (seq, key) = k_base[seq] + key
+    float* S;                // score of launch row r, key s at S[r * ld_s + s]
+    int64_t ld_s;
+    uint32_t* status;
+    int32_t n_stages;
+    int32_t pad_;
+};
+
+template <int D, int H>
+struct TcShape {
+    static constexpr int NQA = 256 / H;                  // queries per accumulator
+    static constexpr int ROWB = D * 2 >= 128 ? 128 : 64;   // swizzle width = bytes of one box row
+    static constexpr int BOXC = ROWB / 2;                 // bf16 elements per box row
+    static constexpr int NBOX = D / BOXC;                 // boxes across d
+    static constexpr int KSTEPS = D / 16;                 // MMAs of K = 16 per tile
+    static constexpr uint32_t QBOX = 256u * ROWB;         // one Q box: 256 rows
+    static constexpr uint32_t QACC = 256u * D * 2;        // Q operand of one accumulator
+    static constexpr uint32_t KBOX = 128u * ROWB;
+    static constexpr uint32_t KTILE = 128u * D * 2;
+    static constexpr uint32_t W_BYTES = 2u * NQA * H * 4;
+    static constexpr uint32_t NC_BYTES = 2u * NQA * 4;
+    static constexpr uint32_t BAR_BYTES = 256;
+
+    __host__ __device__ static uint32_t smem_bytes(int n_acc, int n_stages)
+    {
+        return n_acc * QACC + n_stages * KTILE + W_BYTES + NC_BYTES + BAR_BYTES;
+    }
+};
+
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, uint32_t* status, uint32_t where,
+                                        volatile int32_t* abort_flag)
+{
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 256; ++i)
+            if (mbar_test(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            record_error(status, kErrWaitTimeout, where);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+template <int D, int H>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, TcArgs a)
+{
+    using SH = TcShape<D, H>;
+    constexpr int NQA = SH::NQA;
+    constexpr int QH = NQA / 2;   // queries of one accumulator handled by one epilogue half
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const TcUnit u = a.units[blockIdx.x];
+    if (u.kt1 <= u.kt0 || u.nrows <= 0) return;   // nothing to score (uniform exit)
+    if (smem_u32(smem) & 1023u) {                 // the swizzled tiles need 1024-byte alignment
+        if (threadIdx.x == 0) record_error(a.status, kErrSmemAlign, blockIdx.x);
+        return;
+    }
+    const int n_acc = u.nrows > NQA ? 2 : 1;
+    const int n_stages = a.n_stages;
+    uint8_t* sQ = smem;
+    uint8_t* sK = smem + n_acc * SH::QACC;
+    float* sW = reinterpret_cast<float*>(sK + n_stages * SH::KTILE);
+    int32_t* sNc = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(sW) + SH::W_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sNc) + SH::NC_BYTES);
+    uint64_t* empty = full + n_stages;
+    uint64_t* qfull = empty + n_stages;
+    uint64_t* tfull = qfull + 1;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < n_stages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(qfull, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 8 * 32);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 512);
+    if (warp >= 2) {   // stage the tile's head weights and eligible counts
+        for (int i = threadIdx.x - 64; i < 2 * NQA * H; i += kTcThreads - 64) {
+            const int j = i / H;
+            sW[i] = j < u.nrows ? a.W[(int64_t)a.rows[u.row0 + j].qrow * H + (i % H)] : 0.f;
+        }
+        for (int j = threadIdx.x - 64; j < 2 * NQA; j += kTcThreads - 64)
+            sNc[j] = j < u.nrows ? a.rows[u.row0 + j].ncols : 0;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const RowDesc first = a.rows[u.row0];
+    const int nkt = u.kt1 - u.kt0;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tmQ);
+            prefetch_tensormap(&tmK);
+            mbar_arrive_expect_tx(qfull, n_acc * SH::QACC);
+            for (int acc = 0; acc < n_acc; ++acc)
+                for (int bx = 0; bx < SH::NBOX; ++bx)
+                    tma_load_2d(sQ + acc * SH::QACC + bx * SH::QBOX, &tmQ, bx * SH::BOXC, (first.qrow + acc * NQA) * H,
+                                qfull);
+            const int krow0 = a.k_base[first.seq];
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            for (int i = 0; i < nkt; ++i) {
+                if (!tc_wait(&empty[stage], phase ^ 1u, a.status, 1, abort_flag)) break;
+                mbar_arrive_expect_tx(&full[stage], SH::KTILE);
+                const int krow = krow0 + (u.kt0 + i) * 128;
+                for (int bx = 0; bx < SH::NBOX; ++bx)
+                    tma_load_2d(sK + stage * SH::KTILE + bx * SH::KBOX, &tmK, bx * SH::BOXC, krow, &full[stage]);
+                ++issued;
+                if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+            }
+            // Before leaving, every copy this thread started must have landed.
+            if (*abort_flag) {
+                mbar_wait(qfull, 0, a.status, 10);
+                for (int back = 1; back <= n_stages && back <= issued; ++back) {
+                    const int i = issued - back;
+                    mbar_wait(&full[i % n_stages], (uint32_t)((i / n_stages) & 1), a.status, 11);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            uint32_t idesc[2];
+            for (int acc = 0; acc < 2; ++acc) {
+                int nq = u.nrows - acc * NQA;
+                nq = nq < NQA ? nq : NQA;
+                int N = ((nq > 0 ? nq : 1) * H + 15) & ~15;
+                idesc[acc] = idesc_bf16_f32(128, N);
+            }
+            if (tc_wait(qfull, 0, a.status, 2, abort_flag)) {
+                tc_fence_after();
+                int stage = 0;
+                uint32_t phase = 0;
+                uint32_t tph[2] = {0, 0};
+                for (int i = 0; i < nkt && !*abort_flag; ++i) {
+                    if (!tc_wait(&full[stage], phase, a.status, 3, abort_flag)) break;
+                    tc_fence_after();
+                    for (int acc = 0; acc < n_acc; ++acc) {
+                        if (!tc_wait(&tempty[acc], tph[acc] ^ 1u, a.status, 4, abort_flag)) break;
+                        tc_fence_after();
+                        const uint32_t d = tmem + acc * 256;
+#pragma unroll
+                        for (int kk = 0; kk < SH::KSTEPS; ++kk) {
+                            const int bx = kk / (SH::BOXC / 16);
+                            const uint32_t ko = (kk % (SH::BOXC / 16)) * 32;
+                            const uint64_t ad =
+                                smem_desc_kmajor(smem_u32(sK + stage * SH::KTILE + bx * SH::KBOX) + ko, SH::ROWB);
+                            const uint64_t bd =
+                                smem_desc_kmajor(smem_u32(sQ + acc * SH::QACC + bx * SH::QBOX) + ko, SH::ROWB);
+                            tc_mma(d, ad, bd, idesc[acc], kk > 0 ? 1u : 0u);
+                        }
+                        tc_commit(&tfull[acc]);
+                        tph[acc] ^= 1u;
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // All MMAs issued by this thread complete before TMEM is released.
+            tc_commit(drain);
+            mbar_wait(drain, 0, a.status, 12);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------- epilogue
+        const int quarter = warp & 3;           // TMEM lanes this warp may read
+        const int half = (warp - 2) >> 2;       // which 128 columns of an accumulator
+        uint32_t tph[2] = {0, 0};
+        for (int i = 0; i < nkt; ++i) {
+            const int key = (u.kt0 + i) * 128 + quarter * 32 + lane;
+            for (int acc = 0; acc < n_acc; ++acc) {
+                if (!tc_wait(&tfull[acc], tph[acc], a.status, 5, abort_flag)) break;
+                tph[acc] ^= 1u;
+                tc_fence_after();
+                float v[128];
+                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + acc * 256 + half * 128;
+                tmem_ld32(taddr, v);
+                tmem_ld32(taddr + 32, v + 32);
+                tmem_ld32(taddr + 64, v + 64);
+                tmem_ld32(taddr + 96, v + 96);
+                tmem_ld_wait();
+                tmem_regs_ready<128>(v);
+                tc_fence_before();
+                mbar_arrive(&tempty[acc]);   // the accumulator may be overwritten from here on
+
+                const int jbase = acc * NQA + half * QH;
+#pragma unroll
+                for (int q = 0; q < QH; ++q) {
+                    const int j = jbase + q;
+                    const float* w = sW + j * H;
+                    float s0 = 0.f, s1 = 0.f;
+                    if constexpr (H % 4 == 0) {
+#pragma unroll
+                        for (int h = 0; h < H; h += 4) {
+                            const float4 w4 = *reinterpret_cast<const float4*>(w + h);
+                            s0 = fmaf(w4.x, fmaxf(v[q * H + h], 0.f), s0);
+                            s1 = fmaf(w4.y, fmaxf(v[q * H + h + 1], 0.f), s1);
+                            s0 = fmaf(w4.z, fmaxf(v[q * H + h + 2], 0.f), s0);
+                            s1 = fmaf(w4.w, fmaxf(v[q * H + h + 3], 0.f), s1);
+                        }
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < H; ++h) s0 = fmaf(w[h], fmaxf(v[q * H + h], 0.f), s0);
+                    }
+                    if (j < u.nrows && key < sNc[j])
+                        a.S[(int64_t)(u.row0 + j) * a.ld_s + key] = (s0 + s1) + 0.f;   // -0 -> +0
+                }
+            }
+            if (*abort_flag) break;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace dsa

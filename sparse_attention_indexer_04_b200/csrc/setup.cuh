@@ -216,4 +216,52 @@ __global__ void hisa_kept_kernel(const RowDesc* block_rows, const int32_t* mid, 
     token_rows[t] = RowDesc{t, br.seq, ncols, t};
 }
 
+// ------------------------------------------------------ tensor-core units
+struct TcUnitOut {
+    int32_t row0, nrows, kt0, kt1;
+};
+
+// Work units of one tensor-core scoring launch over launch rows
+// [0, n_rows) = absolute rows [row_base, row_base + n_rows).  Rows are cut into
+// tiles of at most TQ consecutive rows of one sequence (seq_off: absolute
+// row offsets per sequence); each tile's key tiles are split `splits` ways.
+// Within a sequence tiles are emitted last-first, so the longest causal
+// tiles start first.  Single CTA; tile_base is [n_seqs + 1] scratch.
+__global__ void tc_units_kernel(const RowDesc* rows, int32_t n_rows, int32_t row_base, const int32_t* seq_off,
+                                int32_t n_seqs, int32_t TQ, int32_t splits, int32_t* tile_base, TcUnitOut* units)
+{
+    if (threadIdx.x == 0) {
+        int32_t acc = 0;
+        for (int b = 0; b < n_seqs; ++b) {
+            tile_base[b] = acc;
+            const int lo = max(seq_off[b], row_base), hi = min(seq_off[b + 1], row_base + n_rows);
+            if (hi > lo) acc += (hi - lo + TQ - 1) / TQ;
+        }
+        tile_base[n_seqs] = acc;
+    }
+    __syncthreads();
+    const int total = tile_base[n_seqs];
+    for (int tau = threadIdx.x; tau < total; tau += blockDim.x) {
+        const int b = find_seq(tile_base, n_seqs, tau);
+        const int lo = max(seq_off[b], row_base), hi = min(seq_off[b + 1], row_base + n_rows);
+        const int ntile = (hi - lo + TQ - 1) / TQ;
+        const int jj = ntile - 1 - (tau - tile_base[b]);
+        const int r0 = lo + jj * TQ - row_base;
+        const int nr = min(TQ, hi - lo - jj * TQ);
+        int maxnc = 0;
+        for (int r = r0; r < r0 + nr; ++r) maxnc = max(maxnc, rows[r].ncols);
+        const int nkt = (maxnc + 127) / 128;
+        for (int s = 0; s < splits; ++s)
+            units[tau * splits + s] = TcUnitOut{r0, nr, nkt * s / splits, nkt * (s + 1) / splits};
+    }
+}
+
+// Fills a row-major [rows, cols] fp32 matrix with -inf (masked scores).
+__global__ void fill_neg_inf_kernel(float* S, int64_t ld, int32_t rows, int32_t cols)
+{
+    const int64_t total = (int64_t)rows * cols;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x)
+        S[(i / cols) * ld + (i % cols)] = -INFINITY;
+}
+
 }  // namespace dsa
