@@ -178,6 +178,28 @@ dsa_status hisa_index(const dsa_batch* batch, const void* Q, const void* K, cons
 dsa_status dsa_device_check(void* ws, void* stream, uint32_t* detail);
 
 /* --------------------------------------------------------------------
+ * Allocation-free dense top-k (no counterpart in the pages; a convenience of
+ * this library).  Same computation, arguments and outputs as dsa_index_topk,
+ * but the workspace is a device array inside the library, for callers that
+ * cannot call cudaMalloc (for example a custom-op callback of an inference
+ * runtime that is given no allocator and must not allocate while it runs).
+ *  - Capacity: dsa_index_topk_static_capacity() bytes (8 MiB), held by every
+ *    GPU that loads the library until the process exits.  A batch whose
+ *    dsa_index_topk_workspace exceeds it is rejected with DSA_ERR_WORKSPACE
+ *    before anything is launched.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array: calls that overlap on the
+ *    GPU (different streams, or different host threads) race and corrupt each
+ *    other's results.  Serialise them.
+ *  - Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ */
+size_t dsa_index_topk_static_capacity(void);
+dsa_status dsa_index_topk_static(const dsa_batch* batch, const void* Q, const void* K, const float* W,
+                                 int32_t k, int32_t* idx, float* scores, void* stream);
+
+/* --------------------------------------------------------------------
  * Launch accounting and kernel timing, for benchmarks (not part of the
  * indexer; no counterpart on the pages).  The only process-wide state of
  * the library.

@@ -70,6 +70,8 @@ _sig("hisa_pool_keys", ctypes.c_int, _B, _P, _I32, _P, _P)
 _sig("hisa_index_workspace", _SZ, _B, _I32, _I32, _I32)
 _sig("hisa_index", ctypes.c_int, _B, _P, _P, _P, _P, _I32, _I32, _I32, _P, _P, _P, _SZ, _P)
 _sig("dsa_device_check", ctypes.c_int, _P, _P, ctypes.POINTER(ctypes.c_uint32))
+_sig("dsa_index_topk_static_capacity", _SZ)
+_sig("dsa_index_topk_static", ctypes.c_int, _B, _P, _P, _P, _I32, _P, _P, _P)
 _sig("dsa_profile_enable", None, _I32)
 _sig("dsa_launch_count", ctypes.c_uint64)
 _sig("dsa_profile_kind_name", ctypes.c_char_p, _I32)
@@ -173,6 +175,22 @@ def index_topk(layout: Layout, Q, K, W, k: int, idx=None, scores=None, want_scor
     _check(_lib.dsa_index_topk(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), k, _ptr(idx), _ptr(scores), _ptr(ws),
                                _bytes(ws), _stream(stream)), "dsa_index_topk")
     return (idx, scores) if want_scores else idx
+
+
+def index_topk_static(layout: Layout, Q, K, W, k: int, idx=None, scores=None, want_scores=False, stream=None):
+    """dsa_index_topk with the library's built-in device scratch instead of a workspace (allocates nothing
+    in the library; for callers that cannot allocate).  Calls on one device must not overlap on the GPU."""
+    if idx is None:
+        idx = torch.empty(layout.num_queries, k, dtype=torch.int32, device=layout.device)
+    if want_scores and scores is None:
+        scores = torch.empty(layout.num_queries, k, dtype=torch.float32, device=layout.device)
+    _check(_lib.dsa_index_topk_static(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), k, _ptr(idx), _ptr(scores),
+                                      _stream(stream)), "dsa_index_topk_static")
+    return (idx, scores) if want_scores else idx
+
+
+def index_topk_static_capacity() -> int:
+    return int(_lib.dsa_index_topk_static_capacity())
 
 
 # ------------------------------------------------------------------- PIVOT

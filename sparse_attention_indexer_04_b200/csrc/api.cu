@@ -791,3 +791,57 @@ dsa_status dsa_device_check(void* ws, void* stream, uint32_t* detail)
 }
 
 }  // extern "C"
+
+// =====================================================================
+// Allocation-free variant of dsa_index_topk.
+//
+// Some callers cannot call cudaMalloc at all: for example an inference
+// runtime's custom-op callback that is handed no allocator and must not
+// allocate while it runs, or a latency-critical loop that is not allowed to
+// touch the device allocator.  For them the workspace of dsa_index_topk lives
+// in this file-scope device array instead of caller memory.  Every GPU that
+// loads the library holds it (kStaticScratchBytes) until the process exits.
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;   // 8 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device with cudaGetSymbolAddress (with that device current) and cached.
+dsa_status static_scratch(void** out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" size_t dsa_index_topk_static_capacity(void) { return kStaticScratchBytes; }
+
+extern "C" dsa_status dsa_index_topk_static(const dsa_batch* b, const void* Q, const void* K, const float* W,
+                                            int32_t k, int32_t* idx, float* scores, void* stream)
+{
+    HostInfo hi;
+    dsa_status s = check_batch(b, &hi);
+    if (s != DSA_OK) return s;
+    if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
+    DensePlan p;
+    if (dense_plan(nullptr, b, hi, false, &p) > kStaticScratchBytes) return DSA_ERR_WORKSPACE;
+    void* ws = nullptr;
+    if ((s = static_scratch(&ws)) != DSA_OK) return s;
+    // dsa_index_topk clears the status word at the start of every call; nothing else must start at zero.
+    return dsa_index_topk(b, Q, K, W, k, idx, scores, ws, kStaticScratchBytes, stream);
+}
