@@ -173,15 +173,11 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
     a.rows = rows; a.n_rows = n_rows; a.k = k; a.map = map; a.S = S; a.ld_s = ld_s;
     a.src_from_list = src_from_list ? 1 : 0;
     a.out_idx = out_idx; a.ld_idx = ld_idx; a.out_score = out_score; a.ld_score = ld_score;
-    if (max_cols <= kSelectSmemKeys) {
-        const size_t smem = size_t(std::max(max_cols, 1)) * sizeof(uint32_t);
-        if (cudaFuncSetAttribute(select_topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(kSelectSmemKeys * sizeof(uint32_t))) != cudaSuccess)
-            return DSA_ERR_CUDA;
-        DSA_LAUNCH(kProfSelect, st, select_topk_kernel<true><<<n_rows, kSelectThreads, smem, st>>>(a));
-    } else {
-        DSA_LAUNCH(kProfSelect, st, select_topk_kernel<false><<<n_rows, kSelectThreads, 0, st>>>(a));
-    }
+    const size_t smem = select_smem_bytes(std::max(max_cols, 1));
+    if (cudaFuncSetAttribute(select_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return DSA_ERR_CUDA;
+    DSA_LAUNCH(kProfSelect, st, select_stream_kernel<<<n_rows, kSelThreads, smem, st>>>(a));
     return launched();
 }
 

@@ -117,3 +117,22 @@ def test_full_size_prefill_32k_sampled_rows():
     counts = (idx >= 0).sum(1)
     assert np.array_equal(counts, np.minimum(np.arange(b.n_q) + 1, 2048))
     assert np.all(idx.max(1) <= np.arange(b.n_q))
+
+
+@pytest.mark.parametrize("sampled_high", [True, False])
+def test_select_when_the_even_sample_misleads(sampled_high):
+    """The top-k picks a threshold from 2048 evenly spaced columns of a long row.  Keys that make exactly
+    those columns score high (too few columns then pass the threshold) or low (too many pass) must still
+    give the exact answer: integer inputs, compared exactly with the oracle."""
+    L, k = 20000, 3000
+    b = workloads.ragged(30, [2], [L], H=1, d=32, k=k, integer=True)
+    sampled = np.unique((np.arange(2048, dtype=np.int64) * (L - 1 + 1)) // 2048)    # n = L for the last query
+    hi, lo = (3.0, 1.0) if sampled_high else (1.0, 3.0)
+    K = np.full((L, 32), lo, np.float32)
+    K[sampled] = hi
+    K[::7, 0] += 1.0                       # some variation, many exact ties remain
+    b.K = torch.as_tensor(K).to(torch.bfloat16)
+    b.Q = torch.ones_like(b.Q)
+    b.W = torch.ones_like(b.W)
+    b.q_pos = torch.tensor([L - 2, L - 1], dtype=torch.int32)
+    exact_topk(b, k)
