@@ -261,7 +261,9 @@ int32_t tc_splits(int32_t tiles, int32_t max_cols)
 }
 
 // A query-row source for the tensor-core path: rows r of the launch read
-// Q[rd.qrow] / W[rd.qrow]; seq_off are absolute row offsets per sequence.
+// Q[rd.qrow] / W[rd.qrow]; seq_off are absolute row offsets of the segments
+// (runs of rows that share one column -> key map: sequences, PIVOT groups or
+// single HISA queries), with a host copy for sizing.
 struct TcSource {
     const void* Q;
     int64_t q_rows;
@@ -284,8 +286,8 @@ int32_t tc_unit_capacity(const TcSource& src, int32_t n_rows, int32_t chunk, int
 }
 
 template <int D, int H>
-dsa_status launch_tc_shape(const CUtensorMap& mq, const CUtensorMap& mk, const TcArgs& a, int32_t n_units,
-                           int n_acc, cudaStream_t st)
+dsa_status launch_tc_shape(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mkg, const TcArgs& a,
+                           int32_t n_units, int n_acc, cudaStream_t st)
 {
     using SH = TcShape<D, H>;
     const int budget = 232448;
@@ -298,41 +300,44 @@ dsa_status launch_tc_shape(const CUtensorMap& mq, const CUtensorMap& mk, const T
     const int smem = std::max((int)SH::smem_bytes(n_acc, stages), 120 * 1024);
     if (cudaFuncSetAttribute(score_tc_kernel<D, H>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return DSA_ERR_CUDA;
-    DSA_LAUNCH(kProfScoreTc, st, score_tc_kernel<D, H><<<n_units, kTcThreads, smem, st>>>(mq, mk, args));
+    DSA_LAUNCH(kProfScoreTc, st, score_tc_kernel<D, H><<<n_units, kTcThreads, smem, st>>>(mq, mk, mkg, args));
     return launched();
 }
 
 template <int D>
-dsa_status launch_tc_d(int H, const CUtensorMap& mq, const CUtensorMap& mk, const TcArgs& a, int32_t n_units,
-                       int n_acc, cudaStream_t st)
+dsa_status launch_tc_d(int H, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mkg, const TcArgs& a,
+                       int32_t n_units, int n_acc, cudaStream_t st)
 {
     switch (H) {
-    case 1: return launch_tc_shape<D, 1>(mq, mk, a, n_units, n_acc, st);
-    case 2: return launch_tc_shape<D, 2>(mq, mk, a, n_units, n_acc, st);
-    case 4: return launch_tc_shape<D, 4>(mq, mk, a, n_units, n_acc, st);
-    case 8: return launch_tc_shape<D, 8>(mq, mk, a, n_units, n_acc, st);
-    case 16: return launch_tc_shape<D, 16>(mq, mk, a, n_units, n_acc, st);
-    case 32: return launch_tc_shape<D, 32>(mq, mk, a, n_units, n_acc, st);
-    default: return launch_tc_shape<D, 64>(mq, mk, a, n_units, n_acc, st);
+    case 1: return launch_tc_shape<D, 1>(mq, mk, mkg, a, n_units, n_acc, st);
+    case 2: return launch_tc_shape<D, 2>(mq, mk, mkg, a, n_units, n_acc, st);
+    case 4: return launch_tc_shape<D, 4>(mq, mk, mkg, a, n_units, n_acc, st);
+    case 8: return launch_tc_shape<D, 8>(mq, mk, mkg, a, n_units, n_acc, st);
+    case 16: return launch_tc_shape<D, 16>(mq, mk, mkg, a, n_units, n_acc, st);
+    case 32: return launch_tc_shape<D, 32>(mq, mk, mkg, a, n_units, n_acc, st);
+    default: return launch_tc_shape<D, 64>(mq, mk, mkg, a, n_units, n_acc, st);
     }
 }
 
 // Tensor-core scores of launch rows [0, n_rows) (absolute [row_base, ...)) into
-// S[r * ld + s] for eligible keys s < rows[r].ncols.
+// S[r * ld + c] for the eligible columns c < rows[r].ncols; column c is key
+// map(c) of the row's sequence.
 dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const TcSource& src, int H, int D,
-                    const void* K, int64_t n_k, const int32_t* k_base, int32_t max_cols, float* S, int64_t ld,
-                    TcUnitOut* units, int32_t* tile_base, uint32_t* status, cudaStream_t st)
+                    const void* K, int64_t n_k, const int32_t* k_base, const ColMap& map, int32_t max_cols, float* S,
+                    int64_t ld, TcUnitOut* units, int32_t* tile_base, uint32_t* status, cudaStream_t st)
 {
     if (n_rows <= 0 || max_cols <= 0 || n_k <= 0) return DSA_OK;
     const int32_t TQ = tc_tile_rows(H);
     const int32_t tiles = tc_count_tiles(src.seq_off_host, src.n_seqs, row_base, n_rows, TQ);
     if (tiles == 0) return DSA_OK;
     const int32_t splits = tc_splits(tiles, max_cols);
-    CUtensorMap mq, mk;
-    if (!make_tile_map(&mq, src.Q, src.q_rows * H, D, 256) || !make_tile_map(&mk, K, n_k, D, 128))
+    const bool gather = map.kind != kMapIdentity || map.offset != 0;
+    CUtensorMap mq, mk, mkg;
+    if (!make_tile_map(&mq, src.Q, src.q_rows * H, D, 256) || !make_tile_map(&mk, K, n_k, D, 128) ||
+        !make_tile_map(&mkg, K, n_k, D, 1))
         return DSA_ERR_CUDA;
-    DSA_LAUNCH(kProfSetup, st, tc_units_kernel<<<1, 256, 0, st>>>(rows, n_rows, row_base, src.seq_off, src.n_seqs,
-                                                                   TQ, splits, tile_base, units));
+    DSA_LAUNCH(kProfSetup, st, tc_units_kernel<<<1, 1024, 0, st>>>(rows, n_rows, row_base, src.seq_off, src.n_seqs,
+                                                                    TQ, splits, tile_base, units));
     dsa_status s = launched();
     if (s != DSA_OK) return s;
     int32_t max_q = 0;
@@ -341,31 +346,32 @@ dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const
     TcArgs a{};
     a.units = reinterpret_cast<const TcUnit*>(units);
     a.rows = rows;
+    a.map = map;
+    a.gather = gather ? 1 : 0;
     a.W = src.W;
     a.k_base = k_base;
     a.S = S;
     a.ld_s = ld;
     a.status = status;
     switch (D) {
-    case 32: return launch_tc_d<32>(H, mq, mk, a, tiles * splits, n_acc, st);
-    case 64: return launch_tc_d<64>(H, mq, mk, a, tiles * splits, n_acc, st);
-    default: return launch_tc_d<128>(H, mq, mk, a, tiles * splits, n_acc, st);
+    case 32: return launch_tc_d<32>(H, mq, mk, mkg, a, tiles * splits, n_acc, st);
+    case 64: return launch_tc_d<64>(H, mq, mk, mkg, a, tiles * splits, n_acc, st);
+    default: return launch_tc_d<128>(H, mq, mk, mkg, a, tiles * splits, n_acc, st);
     }
 }
 
 // Tensor-core scoring then exact top-k, in row chunks that fit the score buffer.
 dsa_status tc_score_and_select(const RowDesc* rows, int32_t n_rows, const TcSource& src, int H, int D, const void* K,
-                               int64_t n_k, const int32_t* k_base, int32_t max_cols, float* Sbuf, TcUnitOut* units,
-                               int32_t* tile_base, uint32_t* status, int32_t k, int32_t* idx, int64_t ld_idx,
-                               float* scores, cudaStream_t st)
+                               int64_t n_k, const int32_t* k_base, const ColMap& map, int32_t max_cols, float* Sbuf,
+                               TcUnitOut* units, int32_t* tile_base, uint32_t* status, int32_t k, int32_t* idx,
+                               int64_t ld_idx, float* scores, cudaStream_t st)
 {
     const int64_t ld = score_ld(max_cols);
     const int32_t chunk = chunk_rows(n_rows, ld);
-    const ColMap map = ColMap{kMapIdentity, 0, 0, 0, nullptr, 0};
     for (int32_t r0 = 0; r0 < n_rows; r0 += chunk) {
         const int32_t nr = std::min(chunk, n_rows - r0);
-        dsa_status s = tc_score(rows + r0, nr, r0, src, H, D, K, n_k, k_base, max_cols, Sbuf, ld, units, tile_base,
-                                status, st);
+        dsa_status s = tc_score(rows + r0, nr, r0, src, H, D, K, n_k, k_base, map, max_cols, Sbuf, ld, units,
+                                tile_base, status, st);
         if (s != DSA_OK) return s;
         s = launch_select(rows + r0, nr, max_cols, k, map, Sbuf, ld, false, idx + int64_t(r0) * ld_idx, ld_idx,
                           scores ? scores + int64_t(r0) * ld_idx : nullptr, ld_idx, st);
@@ -417,6 +423,7 @@ struct PivotPlan {
     float* S;
     TcUnitOut* units;
     int32_t* tile_base;
+    int32_t* group_rows;   // [n_groups + 1] first query row of each group
 };
 
 int32_t count_groups(const dsa_batch* b, int32_t G)
@@ -433,6 +440,16 @@ std::vector<int32_t> group_offsets_host(const dsa_batch* b, int32_t G)
     std::vector<int32_t> off(b->num_seqs + 1, 0);
     for (int i = 0; i < b->num_seqs; ++i)
         off[i + 1] = off[i] + (b->q_offsets_host[i + 1] - b->q_offsets_host[i] + G - 1) / G;
+    return off;
+}
+
+// Host copy of the query-row offsets of every group (what group_row_offsets_kernel writes).
+std::vector<int32_t> group_rows_host(const dsa_batch* b, int32_t G)
+{
+    std::vector<int32_t> off;
+    for (int i = 0; i < b->num_seqs; ++i)
+        for (int32_t r = b->q_offsets_host[i]; r < b->q_offsets_host[i + 1]; r += G) off.push_back(r);
+    off.push_back(b->num_queries);
     return off;
 }
 
@@ -455,8 +472,14 @@ size_t pivot_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t G,
     p->S = c.take<float>(std::max(s_scan, s_ref));
     const std::vector<int32_t> goff = group_offsets_host(b, G);
     const TcSource src{nullptr, 0, nullptr, nullptr, goff.data(), b->num_seqs};
-    p->units = c.take<TcUnitOut>(tc_unit_capacity(src, count_groups(b, G), chunk_scan, b->num_heads, hi.max_k));
-    p->tile_base = c.take<int32_t>(b->num_seqs + 1);
+    const std::vector<int32_t> groff = group_rows_host(b, G);
+    const TcSource srf{nullptr, 0, nullptr, nullptr, groff.data(), (int32_t)groff.size() - 1};
+    const int32_t cap = std::max(tc_unit_capacity(src, count_groups(b, G), chunk_scan, b->num_heads, hi.max_k),
+                                 tc_unit_capacity(srf, b->num_queries, chunk_rows(std::max(1, b->num_queries), ld_ref),
+                                                  b->num_heads, C));
+    p->units = c.take<TcUnitOut>(cap);
+    p->tile_base = c.take<int32_t>(std::max(b->num_seqs, ng) + 1);
+    p->group_rows = c.take<int32_t>(ng + 1);
     return c.off;
 }
 
@@ -467,7 +490,17 @@ struct HisaPlan {
     int32_t* mid;
     int32_t* kept;
     float* S;
+    int32_t* query_off;    // [n_q + 1] 0..n_q: every query is its own segment
+    TcUnitOut* units;
+    int32_t* tile_base;
 };
+
+std::vector<int32_t> iota_host(int32_t n)
+{
+    std::vector<int32_t> v(n + 1);
+    for (int32_t i = 0; i <= n; ++i) v[i] = i;
+    return v;
+}
 
 size_t hisa_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t B, int32_t keep, HisaPlan* p)
 {
@@ -483,6 +516,12 @@ size_t hisa_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t B, 
     const size_t s_blk = size_t(chunk_rows(nq, ld_blk)) * ld_blk;
     const size_t s_tok = size_t(chunk_rows(nq, ld_tok)) * ld_tok;
     p->S = c.take<float>(std::max(s_blk, s_tok));
+    p->query_off = c.take<int32_t>(nq + 1);
+    const std::vector<int32_t> qoff = iota_host(b->num_queries);
+    const TcSource src{nullptr, 0, nullptr, nullptr, qoff.data(), b->num_queries};
+    p->units = c.take<TcUnitOut>(tc_unit_capacity(src, b->num_queries, chunk_rows(nq, ld_tok), b->num_heads,
+                                                  (keep + 2) * B));
+    p->tile_base = c.take<int32_t>(nq + 1);
     return c.off;
 }
 
@@ -540,7 +579,8 @@ dsa_status dsa_index_scores(const dsa_batch* b, const void* Q, const void* K, co
     DSA_LAUNCH(kProfFill, st, fill_neg_inf_kernel<<<1184, 256, 0, st>>>(S, ld_s, b->num_queries, (int32_t)ld_s));
     if ((s = launched()) != DSA_OK) return s;
     const TcSource src{Q, b->num_queries, W, b->q_offsets, b->q_offsets_host, b->num_seqs};
-    return tc_score(p.rows, b->num_queries, 0, src, b->num_heads, b->head_dim, K, b->num_keys, b->k_offsets, hi.max_k,
+    return tc_score(p.rows, b->num_queries, 0, src, b->num_heads, b->head_dim, K, b->num_keys, b->k_offsets, ColMap{},
+                    hi.max_k,
                     S, ld_s, p.units, p.tile_base, static_cast<uint32_t*>(ws), st);
 }
 
@@ -573,7 +613,7 @@ dsa_status dsa_index_topk(const dsa_batch* b, const void* Q, const void* K, cons
     if ((s = launched()) != DSA_OK) return s;
     const TcSource src{Q, b->num_queries, W, b->q_offsets, b->q_offsets_host, b->num_seqs};
     return tc_score_and_select(p.rows, b->num_queries, src, b->num_heads, b->head_dim, K, b->num_keys, b->k_offsets,
-                               hi.max_k, p.S, p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, scores, st);
+                               ColMap{}, hi.max_k, p.S, p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, scores, st);
 }
 
 // ------------------------------------------------------------------ PIVOT
@@ -625,7 +665,7 @@ dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, c
     // Shared scan: each proxy against its prefix, top-C kept with their proxy scores.
     const std::vector<int32_t> goff = group_offsets_host(b, G);
     const TcSource src{p.Qp, ng, p.Wp, p.group_base, goff.data(), b->num_seqs};
-    s = tc_score_and_select(p.proxy_rows, ng, src, H, D, K, b->num_keys, b->k_offsets, hi.max_k, p.S, p.units,
+    s = tc_score_and_select(p.proxy_rows, ng, src, H, D, K, b->num_keys, b->k_offsets, ColMap{}, hi.max_k, p.S, p.units,
                             p.tile_base, static_cast<uint32_t*>(ws), C, cand, C, p.cand_score, st);
     if (s != DSA_OK) return s;
     DSA_LAUNCH(kProfSetup, st, pivot_query_rows_kernel<<<(b->num_queries + 255) / 256, 256, 0, st>>>(
@@ -639,10 +679,15 @@ dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, c
         // Reuse: rank the group's candidates by their proxy scores inside each query's prefix.
         return launch_select(p.query_rows, b->num_queries, C, k, m, p.cand_score, C, true, idx, k, nullptr, 0, st);
     }
-    // Refine: each query scores its eligible candidates with its own indexer.
-    return score_and_select<__nv_bfloat16>(p.query_rows, b->num_queries, C, m, Q, W, H, D,
-                                           static_cast<const __nv_bfloat16*>(K), b->k_offsets, p.S, k, idx, k,
-                                           nullptr, st);
+    // Refine: each query scores its eligible candidates with its own indexer (tensor cores,
+    // the group's candidate keys gathered tile by tile).
+    DSA_LAUNCH(kProfSetup, st, group_row_offsets_kernel<<<(ng + 256) / 256, 256, 0, st>>>(p.groups, ng, b->num_queries,
+                                                                                          p.group_rows));
+    if ((s = launched()) != DSA_OK) return s;
+    const std::vector<int32_t> groff = group_rows_host(b, G);
+    const TcSource srf{Q, b->num_queries, W, p.group_rows, groff.data(), ng};
+    return tc_score_and_select(p.query_rows, b->num_queries, srf, H, D, K, b->num_keys, b->k_offsets, m, C, p.S,
+                               p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, nullptr, st);
 }
 
 // ------------------------------------------------------------------- HISA
@@ -725,9 +770,12 @@ dsa_status hisa_index(const dsa_batch* b, const void* Q, const void* K, const fl
     m.block = B;
     m.list = kept;
     m.list_ld = keep + 2;
-    return score_and_select<__nv_bfloat16>(p.token_rows, nq, (keep + 2) * B, m, Q, W, H, D,
-                                           static_cast<const __nv_bfloat16*>(K), b->k_offsets, p.S, k, idx, k,
-                                           nullptr, st);
+    DSA_LAUNCH(kProfSetup, st, iota_kernel<<<(nq + 256) / 256, 256, 0, st>>>(p.query_off, nq));
+    if ((s = launched()) != DSA_OK) return s;
+    const std::vector<int32_t> qoff = iota_host(nq);
+    const TcSource src{Q, nq, W, p.query_off, qoff.data(), nq};
+    return tc_score_and_select(p.token_rows, nq, src, H, D, K, b->num_keys, b->k_offsets, m, (keep + 2) * B, p.S,
+                               p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, nullptr, st);
 }
 
 // ---------------------------------------------------------------- profiling

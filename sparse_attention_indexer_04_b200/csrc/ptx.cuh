@@ -93,6 +93,19 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// 2-D gather of four rows (row indices y0..y3, one-row box starting at column
+// c0) into 4 consecutive box rows at dst, completion counted on `bar`.  No multicast.
+__device__ __forceinline__ void tma_gather4_2d(void* dst, const CUtensorMap* map, int32_t c0, int32_t y0, int32_t y1,
+                                               int32_t y2, int32_t y3, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
+          "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

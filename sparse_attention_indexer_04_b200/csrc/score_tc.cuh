@@ -10,8 +10,13 @@
 // cross-thread traffic.
 //
 // A CTA owns one work unit: up to 2 * (256 / H) consecutive queries of one
-// sequence (two accumulators of 256 TMEM columns each, so every key tile in
-// shared memory feeds two MMAs) and a range of its key tiles.  Roles:
+// segment (rows sharing one ordered set of candidate keys: a sequence's
+// prefix, a PIVOT group's candidates, a HISA query's kept blocks) — two
+// accumulators of 256 TMEM columns each, so every key tile in shared memory
+// feeds two MMAs — and a range of its key tiles.  Column c of the segment is
+// key map(c): contiguous key tiles are loaded with TMA tile loads, gathered
+// ones with TMA gather4 (four rows per instruction, one per producer lane).
+// Roles:
 //   warp 0      TMA producer: the query tile once, then a ring of key tiles
 //   warp 1      TMEM allocator and MMA issuer (one thread)
 //   warps 2..9  epilogue: TMEM -> registers, ReLU, weighted head sum, causal
@@ -40,6 +45,10 @@ struct TcUnit {
 struct TcArgs {
     const TcUnit* units;
     const RowDesc* rows;
+    ColMap map;              // column -> key index; identity: contiguous key tiles (TMA tile loads),
+                             // otherwise each tile's 128 keys are gathered (TMA gather4)
+    int32_t gather;          // 0: contiguous tiles, 1: gathered rows
+    int32_t pad2_;
     const float* W;          // row rd.qrow: [H]
     const int32_t* k_base;   // key row of (seq, key) = k_base[seq] + key
     float* S;                // score of launch row r, key s at S[r * ld_s + s]
@@ -90,7 +99,8 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, uint32_t
 
 template <int D, int H>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, TcArgs a)
+    score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmKg, TcArgs a)
 {
     using SH = TcShape<D, H>;
     constexpr int NQA = SH::NQA;
@@ -151,36 +161,54 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
+        const int krow0 = a.k_base[first.seq];
         if (lane == 0) {
             prefetch_tensormap(&tmQ);
-            prefetch_tensormap(&tmK);
+            prefetch_tensormap(a.gather ? &tmKg : &tmK);
             mbar_arrive_expect_tx(qfull, n_acc * SH::QACC);
             for (int acc = 0; acc < n_acc; ++acc)
                 for (int bx = 0; bx < SH::NBOX; ++bx)
                     tma_load_2d(sQ + acc * SH::QACC + bx * SH::QBOX, &tmQ, bx * SH::BOXC, (first.qrow + acc * NQA) * H,
                                 qfull);
-            const int krow0 = a.k_base[first.seq];
-            int stage = 0;
-            uint32_t phase = 0;
-            int issued = 0;
-            for (int i = 0; i < nkt; ++i) {
-                if (!tc_wait(&empty[stage], phase ^ 1u, a.status, 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&full[stage], SH::KTILE);
-                const int krow = krow0 + (u.kt0 + i) * 128;
-                for (int bx = 0; bx < SH::NBOX; ++bx)
-                    tma_load_2d(sK + stage * SH::KTILE + bx * SH::KBOX, &tmK, bx * SH::BOXC, krow, &full[stage]);
-                ++issued;
-                if (++stage == n_stages) { stage = 0; phase ^= 1u; }
-            }
-            // Before leaving, every copy this thread started must have landed.
-            if (*abort_flag) {
-                mbar_wait(qfull, 0, a.status, 10);
-                for (int back = 1; back <= n_stages && back <= issued; ++back) {
-                    const int i = issued - back;
-                    mbar_wait(&full[i % n_stages], (uint32_t)((i / n_stages) & 1), a.status, 11);
+        }
+        int ncmax = 0;   // columns of the unit that exist (tiles past it read column 0's key)
+        for (int j = 0; j < u.nrows; ++j) ncmax = max(ncmax, sNc[j]);
+        int stage = 0;
+        uint32_t phase = 0;
+        int issued = 0;
+        for (int i = 0; i < nkt; ++i) {
+            int ok = 1;
+            if (lane == 0) ok = tc_wait(&empty[stage], phase ^ 1u, a.status, 1, abort_flag) ? 1 : 0;
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (lane == 0) mbar_arrive_expect_tx(&full[stage], SH::KTILE);
+            if (!a.gather) {
+                if (lane == 0) {
+                    const int krow = krow0 + (u.kt0 + i) * 128;
+                    for (int bx = 0; bx < SH::NBOX; ++bx)
+                        tma_load_2d(sK + stage * SH::KTILE + bx * SH::KBOX, &tmK, bx * SH::BOXC, krow, &full[stage]);
                 }
+            } else {
+                __syncwarp();
+                const int c0 = (u.kt0 + i) * 128 + 4 * lane;   // this lane's four rows of the tile
+                int y[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) y[e] = krow0 + map_col(a.map, first, c0 + e < ncmax ? c0 + e : 0);
+                for (int bx = 0; bx < SH::NBOX; ++bx)
+                    tma_gather4_2d(sK + stage * SH::KTILE + bx * SH::KBOX + 4 * lane * SH::ROWB, &tmKg, bx * SH::BOXC,
+                                   y[0], y[1], y[2], y[3], &full[stage]);
+            }
+            ++issued;
+            if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+        }
+        // Before leaving, every copy this warp started must have landed.
+        if (lane == 0 && *abort_flag) {
+            mbar_wait(qfull, 0, a.status, 10);
+            for (int back = 1; back <= n_stages && back <= issued; ++back) {
+                const int i = issued - back;
+                mbar_wait(&full[i % n_stages], (uint32_t)((i / n_stages) & 1), a.status, 11);
             }
         }
+        __syncwarp();
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer
         if (lane == 0) {

@@ -223,27 +223,42 @@ struct TcUnitOut {
 
 // Work units of one tensor-core scoring launch over launch rows
 // [0, n_rows) = absolute rows [row_base, row_base + n_rows).  Rows are cut into
-// tiles of at most TQ consecutive rows of one sequence (seq_off: absolute
-// row offsets per sequence); each tile's key tiles are split `splits` ways.
-// Within a sequence tiles are emitted last-first, so the longest causal
-// tiles start first.  Single CTA; tile_base is [n_seqs + 1] scratch.
-__global__ void tc_units_kernel(const RowDesc* rows, int32_t n_rows, int32_t row_base, const int32_t* seq_off,
-                                int32_t n_seqs, int32_t TQ, int32_t splits, int32_t* tile_base, TcUnitOut* units)
+// tiles of at most TQ consecutive rows of one segment (seg_off: absolute row
+// offsets per segment); each tile's key tiles are split `splits` ways.
+// Within a segment tiles are emitted last-first, so the longest causal tiles
+// start first.  One CTA of 1024 threads; tile_base is [n_seg + 1] scratch.
+__global__ void tc_units_kernel(const RowDesc* rows, int32_t n_rows, int32_t row_base, const int32_t* seg_off,
+                                int32_t n_seg, int32_t TQ, int32_t splits, int32_t* tile_base, TcUnitOut* units)
 {
-    if (threadIdx.x == 0) {
-        int32_t acc = 0;
-        for (int b = 0; b < n_seqs; ++b) {
-            tile_base[b] = acc;
-            const int lo = max(seq_off[b], row_base), hi = min(seq_off[b + 1], row_base + n_rows);
-            if (hi > lo) acc += (hi - lo + TQ - 1) / TQ;
-        }
-        tile_base[n_seqs] = acc;
-    }
+    __shared__ int32_t part[1024];
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int per = (n_seg + nt - 1) / nt;   // contiguous segments per thread
+    const int s0 = min(n_seg, tid * per), s1 = min(n_seg, s0 + per);
+    auto tiles_of = [&](int b) {
+        const int lo = max(seg_off[b], row_base), hi = min(seg_off[b + 1], row_base + n_rows);
+        return hi > lo ? (hi - lo + TQ - 1) / TQ : 0;
+    };
+    int sum = 0;
+    for (int b = s0; b < s1; ++b) sum += tiles_of(b);
+    part[tid] = sum;
     __syncthreads();
-    const int total = tile_base[n_seqs];
-    for (int tau = threadIdx.x; tau < total; tau += blockDim.x) {
-        const int b = find_seq(tile_base, n_seqs, tau);
-        const int lo = max(seq_off[b], row_base), hi = min(seq_off[b + 1], row_base + n_rows);
+    for (int o = 1; o < nt; o <<= 1) {   // inclusive scan of the per-thread sums
+        const int x = tid >= o ? part[tid - o] : 0;
+        __syncthreads();
+        part[tid] += x;
+        __syncthreads();
+    }
+    int acc = part[tid] - sum;
+    for (int b = s0; b < s1; ++b) {
+        tile_base[b] = acc;
+        acc += tiles_of(b);
+    }
+    if (tid == nt - 1) tile_base[n_seg] = part[nt - 1];
+    __syncthreads();
+    const int total = tile_base[n_seg];
+    for (int tau = tid; tau < total; tau += nt) {
+        const int b = find_seq(tile_base, n_seg, tau);
+        const int lo = max(seg_off[b], row_base), hi = min(seg_off[b + 1], row_base + n_rows);
         const int ntile = (hi - lo + TQ - 1) / TQ;
         const int jj = ntile - 1 - (tau - tile_base[b]);
         const int r0 = lo + jj * TQ - row_base;
@@ -254,6 +269,21 @@ __global__ void tc_units_kernel(const RowDesc* rows, int32_t n_rows, int32_t row
         for (int s = 0; s < splits; ++s)
             units[tau * splits + s] = TcUnitOut{r0, nr, nkt * s / splits, nkt * (s + 1) / splits};
     }
+}
+
+// Row offsets of PIVOT groups (segment g = rows [off[g], off[g+1])) and of
+// single-query segments (off[t] = t), for the tensor-core unit builder.
+__global__ void group_row_offsets_kernel(const GroupDesc* groups, int32_t n_groups, int32_t n_q, int32_t* off)
+{
+    const int g = blockIdx.x * blockDim.x + threadIdx.x;
+    if (g < n_groups) off[g] = groups[g].first;
+    if (g == 0) off[n_groups] = n_q;
+}
+
+__global__ void iota_kernel(int32_t* off, int32_t n)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i <= n) off[i] = i;
 }
 
 // Fills a row-major [rows, cols] fp32 matrix with -inf (masked scores).
