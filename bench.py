@@ -245,6 +245,12 @@ def secondary(device, flush, steps):
             ms = time_steps(step, steps, flush)
             r = {"us_per_step": round(1e3 * sum(ms) / steps, 2), "steps": steps, "setup_s": round(time.time() - t0, 1)}
             r.update(extra(step, sum(ms) / steps))
+            step.dsa.profile_enable(True)                      # a second, separately timed pass per kernel
+            time_steps(step, steps, flush)
+            prof = step.dsa.profile_read()
+            step.dsa.profile_enable(False)
+            r["kernels_us_per_step"] = {k: round(1e3 * v[0] / steps, 2) for k, v in prof.items()}
+            r["launches_per_step"] = sum(v[1] for v in prof.values()) / steps
             out[name] = r
             del step
             torch.cuda.empty_cache()

@@ -173,7 +173,12 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
     a.rows = rows; a.n_rows = n_rows; a.k = k; a.map = map; a.S = S; a.ld_s = ld_s;
     a.src_from_list = src_from_list ? 1 : 0;
     a.out_idx = out_idx; a.ld_idx = ld_idx; a.out_score = out_score; a.ld_score = ld_score;
-    const size_t smem = select_smem_bytes(std::max(max_cols, 1));
+    // Candidate buffer: 1.75 k entries, or what fits next to the bitmaps (a smaller buffer only
+    // sends more rows down the exact full-row path).
+    const size_t fixed = select_smem_bytes(std::max(max_cols, 1), 0) + 2048;
+    const int fit = (int)(((size_t)227 * 1024 - fixed) / 8) & ~255;
+    a.buf_cap = std::max(256, std::min(select_buf_cap(k), fit));
+    const size_t smem = select_smem_bytes(std::max(max_cols, 1), a.buf_cap);
     if (cudaFuncSetAttribute(select_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return DSA_ERR_CUDA;

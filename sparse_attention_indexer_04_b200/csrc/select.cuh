@@ -8,9 +8,9 @@
 // are in flight per SM:
 //   1. threshold: the keys of 2048 evenly spaced columns are ranked and the
 //      one at rank k*m/n plus a 4-sigma margin becomes tau (rows with at most
-//      kBufCap columns skip this and keep every column);
+//      select_buf_cap(k) columns skip this and keep every column);
 //   2. one streaming pass appends every column with key >= tau to a
-//      shared-memory buffer (kBufCap entries);
+//      shared-memory buffer (select_buf_cap(k) entries);
 //   3. if at least k columns passed and none was dropped, the top k of the
 //      row are exactly the top k of the buffer: an 8-bit radix select over
 //      the buffer finds T and the number of T-ties to take.  Otherwise
@@ -26,7 +26,13 @@ namespace dsa {
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSampleMax = 2048;
-constexpr int kBufCap = 4096;
+
+// Candidate buffer entries for top-k: at least 4096 and 1.75 k.
+__host__ __device__ inline int select_buf_cap(int k)
+{
+    const int c = (7 * k / 4 + 255) & ~255;
+    return c < 4096 ? 4096 : c;
+}
 
 struct SelectArgs {
     const RowDesc* rows;
@@ -36,7 +42,7 @@ struct SelectArgs {
     const float* S;          // score row r at S + src_row * ld_s
     int64_t ld_s;
     int32_t src_from_list;   // 1: the score row is rows[r].list instead of r
-    int32_t pad_;
+    int32_t buf_cap;         // candidate buffer entries (select_stream_kernel)
     int32_t* out_idx;        // [n_rows, ld_idx]
     int64_t ld_idx;
     float* out_score;        // nullable, [n_rows, ld_score]
@@ -45,10 +51,10 @@ struct SelectArgs {
 
 
 // Dynamic shared memory of select_stream_kernel for rows of up to max_cols columns.
-__host__ __device__ inline size_t select_smem_bytes(int max_cols)
+__host__ __device__ inline size_t select_smem_bytes(int max_cols, int buf_cap)
 {
     const size_t words = (size_t)(max_cols + 31) / 32;
-    return kSampleMax * 4 + kBufCap * 8 + 2 * words * 4;
+    return kSampleMax * 4 + (size_t)buf_cap * 8 + 2 * words * 4;
 }
 
 // Exact rank selection among `count` keys given by get(i): returns the key T
@@ -121,8 +127,9 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(SelectArgs a
 {
     extern __shared__ __align__(16) uint8_t sel_smem[];
     uint32_t* sample = reinterpret_cast<uint32_t*>(sel_smem);
+    const int kBufCap = a.buf_cap;
     uint64_t* buf = reinterpret_cast<uint64_t*>(sel_smem + kSampleMax * 4);
-    uint32_t* gtmap = reinterpret_cast<uint32_t*>(sel_smem + kSampleMax * 4 + kBufCap * 8);
+    uint32_t* gtmap = reinterpret_cast<uint32_t*>(sel_smem + kSampleMax * 4 + (size_t)kBufCap * 8);
     __shared__ uint32_t hist[256];
     __shared__ uint32_t scratch[2 * kSelWarps + 2];
     __shared__ uint32_t s_count;
