@@ -164,6 +164,11 @@ dsa_status launch_score(const RowDesc* rows, int32_t n_rows, int32_t max_cols, c
     return launched();
 }
 
+// Threads per row of the streaming select: 256 when rows fill the GPU several times over, 512
+// when there are few rows (each row's phases are latency-bound).  Measured on the 32K prefill
+// (32768 rows: 256 best) and the 16 x 32K decode (32 rows: 512 best).
+int select_threads(int32_t n_rows) { return n_rows < 2 * 148 ? 512 : 256; }
+
 dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, int32_t k, const ColMap& map,
                          const float* S, int64_t ld_s, bool src_from_list, int32_t* out_idx, int64_t ld_idx,
                          float* out_score, int64_t ld_score, cudaStream_t st)
@@ -179,10 +184,27 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
     const int fit = (int)(((size_t)227 * 1024 - fixed) / 8) & ~255;
     a.buf_cap = std::max(256, std::min(select_buf_cap(k), fit));
     const size_t smem = select_smem_bytes(std::max(max_cols, 1), a.buf_cap);
-    if (cudaFuncSetAttribute(select_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return DSA_ERR_CUDA;
-    DSA_LAUNCH(kProfSelect, st, select_stream_kernel<<<n_rows, kSelThreads, smem, st>>>(a));
+    const int nt = select_threads(n_rows);
+    switch (nt) {
+    case 1024:
+        if (cudaFuncSetAttribute(select_stream_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return DSA_ERR_CUDA;
+        DSA_LAUNCH(kProfSelect, st, select_stream_kernel<1024><<<n_rows, 1024, smem, st>>>(a));
+        break;
+    case 512:
+        if (cudaFuncSetAttribute(select_stream_kernel<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return DSA_ERR_CUDA;
+        DSA_LAUNCH(kProfSelect, st, select_stream_kernel<512><<<n_rows, 512, smem, st>>>(a));
+        break;
+    default:
+        if (cudaFuncSetAttribute(select_stream_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return DSA_ERR_CUDA;
+        DSA_LAUNCH(kProfSelect, st, select_stream_kernel<256><<<n_rows, 256, smem, st>>>(a));
+        break;
+    }
     return launched();
 }
 

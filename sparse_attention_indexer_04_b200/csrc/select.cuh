@@ -62,9 +62,11 @@ __host__ __device__ inline size_t select_smem_bytes(int max_cols, int buf_cap)
 // that rank reaches.  Digits are taken from (key - min), starting at the
 // highest bit where min and max differ, 8 bits at a time, so even the first
 // pass spreads the keys over many bins.  All threads call it.
-template <typename Get>
+template <int NT, typename Get>
 __device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, uint32_t* hist, uint32_t* scratch)
 {
+    constexpr int kSelThreads = NT;
+    constexpr int kSelWarps = NT / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t lo = 0xffffffffu, hi = 0u;
     for (int i = tid; i < count; i += kSelThreads) {
@@ -123,8 +125,11 @@ __device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, 
     return lo + prefix;
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_stream_kernel(SelectArgs a)
+template <int NT>
+__global__ void __launch_bounds__(NT) select_stream_kernel(SelectArgs a)
 {
+    constexpr int kSelThreads = NT;
+    constexpr int kSelWarps = NT / 32;
     extern __shared__ __align__(16) uint8_t sel_smem[];
     uint32_t* sample = reinterpret_cast<uint32_t*>(sel_smem);
     const int kBufCap = a.buf_cap;
@@ -164,7 +169,7 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(SelectArgs a
             int rank = (int)ceilf(expect + 4.f * sqrtf(expect) + 4.f);
             rank = min(rank, m);
             __syncthreads();
-            tau = radix_select([&](int i) { return sample[i]; }, m, rank, hist, scratch);
+            tau = radix_select<NT>([&](int i) { return sample[i]; }, m, rank, hist, scratch);
         }
         // ---- 2. one pass: every column with key >= tau into the buffer
         if (tid == 0) s_count = 0;
@@ -219,7 +224,7 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(SelectArgs a
         krem = k;
         if (count >= k && count <= kBufCap) {
             // ---- 3. exact top-k of the buffer
-            thresh = radix_select([&](int i) { return (uint32_t)(buf[i] >> 32); }, count, krem, hist, scratch);
+            thresh = radix_select<NT>([&](int i) { return (uint32_t)(buf[i] >> 32); }, count, krem, hist, scratch);
             for (int i = tid; i < count; i += kSelThreads) {
                 const uint32_t u = (uint32_t)(buf[i] >> 32), c = (uint32_t)buf[i];
                 if (u > thresh) atomicOr(&gtmap[c >> 5], 1u << (c & 31));
@@ -227,7 +232,7 @@ __global__ void __launch_bounds__(kSelThreads) select_stream_kernel(SelectArgs a
             }
         } else {
             // ---- 3'. the sample misled: exact selection over the whole row
-            thresh = radix_select([&](int i) { return score_key(__ldg(src + i)); }, n, krem, hist, scratch);
+            thresh = radix_select<NT>([&](int i) { return score_key(__ldg(src + i)); }, n, krem, hist, scratch);
             for (int c = tid; c < n; c += kSelThreads) {
                 const uint32_t u = score_key(__ldg(src + c));
                 if (u > thresh) atomicOr(&gtmap[c >> 5], 1u << (c & 31));
