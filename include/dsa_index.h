@@ -35,9 +35,11 @@
  *  Output rows.  Every index row holds min(k, #eligible) sequence-local key
  *  indices in ASCENDING index order, then -1 padding up to k.  Optional
  *  score outputs hold the fp32 score of each returned index (NaN padding).
- *  Supported shapes.  H in {1..64} with H*d*2 a multiple of 16; d in
- *  {32, 64, 128}; 1 <= k <= 16384; per-sequence key count < 2^31.
- *  Otherwise DSA_ERR_UNSUPPORTED.
+ *  Supported shapes.  H a power of two in 1..64; d in {32, 64, 128};
+ *  1 <= k <= 16384; a ranked row (a sequence's keys for the dense top-k and
+ *  PIVOT's proxy scan, its middle blocks for HISA's block filter) of at most
+ *  about 760,000 columns: the selection keeps two bitmaps of the row's
+ *  columns in shared memory.  Otherwise DSA_ERR_UNSUPPORTED.
  *  Ownership.  The caller owns every buffer: inputs, outputs and the
  *  workspace.  The library allocates no device memory, never synchronises
  *  the stream (dsa_device_check and dsa_profile_read excepted) and keeps no

@@ -26,10 +26,17 @@ constexpr size_t kScoreBudget = size_t(256) << 20;   // bytes of materialised sc
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace header: the status word (kStatusBytes), then two counters per row of the split-row
+// select (kSplitMaxRows rows).  Each call clears the header once before its first launch.
+constexpr int32_t kSplitMaxRows = 512;
+constexpr size_t kHeaderBytes = kStatusBytes + size_t(kSplitMaxRows) * 2 * sizeof(uint32_t);
+
+uint32_t* split_counters(void* ws) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + kStatusBytes); }
+
 // Sequential carve-out of a workspace; a dry run (base == nullptr) sizes it.
 struct Carver {
     char* base;
-    size_t off = kStatusBytes;
+    size_t off = kHeaderBytes;
     template <typename T>
     T* take(size_t count)
     {
@@ -169,39 +176,76 @@ dsa_status launch_score(const RowDesc* rows, int32_t n_rows, int32_t max_cols, c
 // (32768 rows: 256 best) and the 16 x 32K decode (32 rows: 512 best).
 int select_threads(int32_t n_rows) { return n_rows < 2 * 148 ? 512 : 256; }
 
+// Candidate buffer entries of the select: 1.75 k, or what fits in shared memory next to the
+// bitmaps of max_cols columns (a smaller buffer only sends more rows down the full-row path).
+int32_t select_cap(int32_t k, int32_t max_cols)
+{
+    const size_t fixed = select_smem_bytes(std::max(max_cols, 1), 0) + 2048;
+    const int fit = (int)(((size_t)227 * 1024 - fixed) / 8) & ~255;
+    return std::max(256, std::min(select_buf_cap(k), fit));
+}
+
+// Whether rows of max_cols columns fit the select's shared memory (sample, a candidate buffer of
+// at least 256 entries, two column bitmaps): up to about 760,000 columns.
+bool select_fits(int32_t k, int32_t max_cols)
+{
+    return select_smem_bytes(std::max(max_cols, 1), select_cap(k, max_cols)) <= (size_t)227 * 1024;
+}
+
+// Scratch of the split-row select: two counters per row in the workspace header (zero between
+// launches) and a global candidate buffer of max_rows x select_cap entries.
+struct SelectSplit {
+    uint32_t* ctr = nullptr;
+    uint64_t* buf = nullptr;
+    int32_t max_rows = 0;
+};
+
+// Rows a plan may hand to the split select in one launch (0: never split).
+int32_t split_rows_for(int32_t chunk) { return chunk <= 2 * 148 ? chunk : 0; }
+
+// CTAs per row of the split select: one wave of at most 148 CTAs over all rows (more CTAs only
+// lengthen the launch ramp; the per-row steps other than the scan do not shrink), each chunk at
+// least 2048 columns (1 = use the one-CTA-per-row kernel).
+int select_parts(int32_t n_rows, int32_t max_cols)
+{
+    if (n_rows <= 0) return 1;
+    return std::max(1, std::min(148 / n_rows, max_cols / 2048));
+}
+
+template <typename Kern>
+dsa_status set_smem(Kern kern, size_t smem)
+{
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess
+               ? DSA_OK
+               : DSA_ERR_CUDA;
+}
+
 dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, int32_t k, const ColMap& map,
                          const float* S, int64_t ld_s, bool src_from_list, int32_t* out_idx, int64_t ld_idx,
-                         float* out_score, int64_t ld_score, cudaStream_t st)
+                         float* out_score, int64_t ld_score, cudaStream_t st, const SelectSplit& sp = SelectSplit{})
 {
     if (n_rows <= 0) return DSA_OK;
     SelectArgs a{};
     a.rows = rows; a.n_rows = n_rows; a.k = k; a.map = map; a.S = S; a.ld_s = ld_s;
     a.src_from_list = src_from_list ? 1 : 0;
     a.out_idx = out_idx; a.ld_idx = ld_idx; a.out_score = out_score; a.ld_score = ld_score;
-    // Candidate buffer: 1.75 k entries, or what fits next to the bitmaps (a smaller buffer only
-    // sends more rows down the exact full-row path).
-    const size_t fixed = select_smem_bytes(std::max(max_cols, 1), 0) + 2048;
-    const int fit = (int)(((size_t)227 * 1024 - fixed) / 8) & ~255;
-    a.buf_cap = std::max(256, std::min(select_buf_cap(k), fit));
+    a.buf_cap = select_cap(k, max_cols);
+    a.sample_bytes = (int32_t)select_sample_bytes(std::max(max_cols, 1));
     const size_t smem = select_smem_bytes(std::max(max_cols, 1), a.buf_cap);
-    const int nt = select_threads(n_rows);
-    switch (nt) {
-    case 1024:
-        if (cudaFuncSetAttribute(select_stream_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-            return DSA_ERR_CUDA;
-        DSA_LAUNCH(kProfSelect, st, select_stream_kernel<1024><<<n_rows, 1024, smem, st>>>(a));
-        break;
+    dsa_status s;
+    const int P = select_parts(n_rows, max_cols);
+    if (sp.buf && sp.ctr && n_rows <= sp.max_rows && P > 1) {
+        if ((s = set_smem(select_split_kernel<512>, smem)) != DSA_OK) return s;
+        DSA_LAUNCH(kProfSelect, st, select_split_kernel<512><<<n_rows * P, 512, smem, st>>>(a, sp.buf, sp.ctr, P));
+        return launched();
+    }
+    switch (select_threads(n_rows)) {
     case 512:
-        if (cudaFuncSetAttribute(select_stream_kernel<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-            return DSA_ERR_CUDA;
+        if ((s = set_smem(select_stream_kernel<512>, smem)) != DSA_OK) return s;
         DSA_LAUNCH(kProfSelect, st, select_stream_kernel<512><<<n_rows, 512, smem, st>>>(a));
         break;
     default:
-        if (cudaFuncSetAttribute(select_stream_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-            return DSA_ERR_CUDA;
+        if ((s = set_smem(select_stream_kernel<256>, smem)) != DSA_OK) return s;
         DSA_LAUNCH(kProfSelect, st, select_stream_kernel<256><<<n_rows, 256, smem, st>>>(a));
         break;
     }
@@ -278,13 +322,22 @@ int32_t tc_count_tiles(const int32_t* off, int n_seqs, int64_t row_base, int64_t
     return (int32_t)n;
 }
 
-// Key-range splits per tile: enough units to fill the GPU twice over when there
-// are few query tiles (decode), each split keeping >= 8 key tiles.
+// Key-range splits per query tile when there are fewer tiles than SMs (decode).
 int32_t tc_splits(int32_t tiles, int32_t max_cols)
 {
     const int32_t kt = (max_cols + 127) / 128;
     if (tiles <= 0 || tiles >= 148 || kt < 16) return 1;
-    return std::max(1, std::min((2 * 148 + tiles - 1) / tiles, kt / 8));
+    // One CTA fills an SM, so the units run in waves of 148: pick the split count s (units of at
+    // least 8 key tiles) minimising waves(s) * (ceil(kt / s) + 2), the 2 standing for a CTA's
+    // start-up (barriers, TMEM, the query tile) in key tiles.
+    int32_t best = 1;
+    int64_t best_cost = INT64_MAX;
+    for (int32_t s = 1; s <= kt / 8; ++s) {
+        const int64_t waves = (int64_t(tiles) * s + 147) / 148;
+        const int64_t cost = waves * ((kt + s - 1) / s + 2);
+        if (cost < best_cost) { best_cost = cost; best = s; }
+    }
+    return best;
 }
 
 // A query-row source for the tensor-core path: rows r of the launch read
@@ -391,7 +444,7 @@ dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const
 dsa_status tc_score_and_select(const RowDesc* rows, int32_t n_rows, const TcSource& src, int H, int D, const void* K,
                                int64_t n_k, const int32_t* k_base, const ColMap& map, int32_t max_cols, float* Sbuf,
                                TcUnitOut* units, int32_t* tile_base, uint32_t* status, int32_t k, int32_t* idx,
-                               int64_t ld_idx, float* scores, cudaStream_t st)
+                               int64_t ld_idx, float* scores, cudaStream_t st, const SelectSplit& sp = SelectSplit{})
 {
     const int64_t ld = score_ld(max_cols);
     const int32_t chunk = chunk_rows(n_rows, ld);
@@ -401,7 +454,7 @@ dsa_status tc_score_and_select(const RowDesc* rows, int32_t n_rows, const TcSour
                                 tile_base, status, st);
         if (s != DSA_OK) return s;
         s = launch_select(rows + r0, nr, max_cols, k, map, Sbuf, ld, false, idx + int64_t(r0) * ld_idx, ld_idx,
-                          scores ? scores + int64_t(r0) * ld_idx : nullptr, ld_idx, st);
+                          scores ? scores + int64_t(r0) * ld_idx : nullptr, ld_idx, st, sp);
         if (s != DSA_OK) return s;
     }
     return DSA_OK;
@@ -422,19 +475,27 @@ struct DensePlan {
     float* S;
     TcUnitOut* units;
     int32_t* tile_base;
+    SelectSplit split;
 };
 
-size_t dense_plan(char* base, const dsa_batch* b, const HostInfo& hi, bool scores_only, DensePlan* p)
+// k = 0: the scores-only entry point (no score buffer, no select).
+size_t dense_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, DensePlan* p)
 {
     Carver c{base};
     const int32_t nq = std::max(1, b->num_queries);
     p->rows = c.take<RowDesc>(nq);
     const int64_t ld = score_ld(hi.max_k);
-    const int32_t chunk = scores_only ? nq : chunk_rows(nq, ld);
+    const int32_t chunk = k == 0 ? nq : chunk_rows(nq, ld);
     const TcSource src{nullptr, 0, nullptr, nullptr, b->q_offsets_host, b->num_seqs};
     p->units = c.take<TcUnitOut>(tc_unit_capacity(src, b->num_queries, chunk, b->num_heads, hi.max_k));
     p->tile_base = c.take<int32_t>(b->num_seqs + 1);
-    if (!scores_only) p->S = c.take<float>(size_t(chunk) * ld);
+    p->split = SelectSplit{};
+    if (k > 0) {
+        p->S = c.take<float>(size_t(chunk) * ld);
+        p->split.max_rows = split_rows_for(chunk);
+        p->split.buf = c.take<uint64_t>(size_t(p->split.max_rows) * select_cap(k, hi.max_k));
+        if (base) p->split.ctr = split_counters(base);
+    }
     return c.off;
 }
 
@@ -520,6 +581,7 @@ struct HisaPlan {
     int32_t* query_off;    // [n_q + 1] 0..n_q: every query is its own segment
     TcUnitOut* units;
     int32_t* tile_base;
+    SelectSplit split;     // the token stage's select
 };
 
 std::vector<int32_t> iota_host(int32_t n)
@@ -529,7 +591,7 @@ std::vector<int32_t> iota_host(int32_t n)
     return v;
 }
 
-size_t hisa_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t B, int32_t keep, HisaPlan* p)
+size_t hisa_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, int32_t B, int32_t keep, HisaPlan* p)
 {
     Carver c{base};
     const int32_t nq = std::max(1, b->num_queries);
@@ -549,13 +611,18 @@ size_t hisa_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t B, 
     p->units = c.take<TcUnitOut>(tc_unit_capacity(src, b->num_queries, chunk_rows(nq, ld_tok), b->num_heads,
                                                   (keep + 2) * B));
     p->tile_base = c.take<int32_t>(nq + 1);
+    p->split = SelectSplit{};
+    p->split.max_rows = split_rows_for(chunk_rows(nq, ld_tok));
+    p->split.buf = c.take<uint64_t>(size_t(p->split.max_rows) * select_cap(k, (keep + 2) * B));
+    if (base) p->split.ctr = split_counters(base);
     return c.off;
 }
 
 dsa_status clear_status(void* ws, cudaStream_t st)
 {
-    return cudaMemsetAsync(ws, 0, kStatusBytes, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+    return cudaMemsetAsync(ws, 0, kHeaderBytes, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
+
 
 }  // namespace
 
@@ -583,7 +650,7 @@ size_t dsa_index_scores_workspace(const dsa_batch* b)
     HostInfo hi;
     if (check_batch(b, &hi) != DSA_OK) return 0;
     DensePlan p;
-    return dense_plan(nullptr, b, hi, true, &p);
+    return dense_plan(nullptr, b, hi, 0, &p);
 }
 
 dsa_status dsa_index_scores(const dsa_batch* b, const void* Q, const void* K, const float* W, float* S,
@@ -595,8 +662,8 @@ dsa_status dsa_index_scores(const dsa_batch* b, const void* Q, const void* K, co
     if ((s = check_tensors(b, Q, K, W)) != DSA_OK) return s;
     if (b->num_queries > 0 && (!S || ld_s < hi.max_k || ld_s > INT32_MAX)) return DSA_ERR_INVALID_ARG;
     DensePlan p;
-    if ((s = check_ws(ws, ws_bytes, dense_plan(nullptr, b, hi, true, &p))) != DSA_OK) return s;
-    dense_plan(static_cast<char*>(ws), b, hi, true, &p);
+    if ((s = check_ws(ws, ws_bytes, dense_plan(nullptr, b, hi, 0, &p))) != DSA_OK) return s;
+    dense_plan(static_cast<char*>(ws), b, hi, 0, &p);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((s = clear_status(ws, st)) != DSA_OK) return s;
     if (b->num_queries == 0) return DSA_OK;
@@ -617,7 +684,7 @@ size_t dsa_index_topk_workspace(const dsa_batch* b, int32_t k)
     HostInfo hi;
     if (check_batch(b, &hi) != DSA_OK || k < 1 || k > kMaxK) return 0;
     DensePlan p;
-    return dense_plan(nullptr, b, hi, false, &p);
+    return dense_plan(nullptr, b, hi, k, &p);
 }
 
 dsa_status dsa_index_topk(const dsa_batch* b, const void* Q, const void* K, const float* W, int32_t k,
@@ -626,12 +693,12 @@ dsa_status dsa_index_topk(const dsa_batch* b, const void* Q, const void* K, cons
     HostInfo hi;
     dsa_status s = check_batch(b, &hi);
     if (s != DSA_OK) return s;
-    if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
+    if (k < 1 || k > kMaxK || !select_fits(k, hi.max_k)) return DSA_ERR_UNSUPPORTED;
     if ((s = check_tensors(b, Q, K, W)) != DSA_OK) return s;
     if (b->num_queries > 0 && !idx) return DSA_ERR_INVALID_ARG;
     DensePlan p;
-    if ((s = check_ws(ws, ws_bytes, dense_plan(nullptr, b, hi, false, &p))) != DSA_OK) return s;
-    dense_plan(static_cast<char*>(ws), b, hi, false, &p);
+    if ((s = check_ws(ws, ws_bytes, dense_plan(nullptr, b, hi, k, &p))) != DSA_OK) return s;
+    dense_plan(static_cast<char*>(ws), b, hi, k, &p);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((s = clear_status(ws, st)) != DSA_OK) return s;
     if (b->num_queries == 0) return DSA_OK;
@@ -640,7 +707,8 @@ dsa_status dsa_index_topk(const dsa_batch* b, const void* Q, const void* K, cons
     if ((s = launched()) != DSA_OK) return s;
     const TcSource src{Q, b->num_queries, W, b->q_offsets, b->q_offsets_host, b->num_seqs};
     return tc_score_and_select(p.rows, b->num_queries, src, b->num_heads, b->head_dim, K, b->num_keys, b->k_offsets,
-                               ColMap{}, hi.max_k, p.S, p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, scores, st);
+                               ColMap{}, hi.max_k, p.S, p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, scores, st,
+                               p.split);
 }
 
 // ------------------------------------------------------------------ PIVOT
@@ -671,7 +739,7 @@ dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, c
     HostInfo hi;
     dsa_status s = check_batch(b, &hi);
     if (s != DSA_OK) return s;
-    if (!pivot_args_ok(k, G, C, mode)) return DSA_ERR_UNSUPPORTED;
+    if (!pivot_args_ok(k, G, C, mode) || !select_fits(C, hi.max_k) || !select_fits(k, C)) return DSA_ERR_UNSUPPORTED;
     if ((s = check_tensors(b, Q, K, W)) != DSA_OK) return s;
     if (b->num_queries > 0 && !idx) return DSA_ERR_INVALID_ARG;
     PivotPlan p;
@@ -754,7 +822,7 @@ size_t hisa_index_workspace(const dsa_batch* b, int32_t k, int32_t B, int32_t ke
     HostInfo hi;
     if (check_batch(b, &hi) != DSA_OK || !hisa_args_ok(k, B, keep)) return 0;
     HisaPlan p;
-    return hisa_plan(nullptr, b, hi, B, keep, &p);
+    return hisa_plan(nullptr, b, hi, k, B, keep, &p);
 }
 
 dsa_status hisa_index(const dsa_batch* b, const void* Q, const void* K, const float* W, const float* pooled,
@@ -764,13 +832,14 @@ dsa_status hisa_index(const dsa_batch* b, const void* Q, const void* K, const fl
     HostInfo hi;
     dsa_status s = check_batch(b, &hi);
     if (s != DSA_OK) return s;
-    if (!hisa_args_ok(k, B, keep)) return DSA_ERR_UNSUPPORTED;
+    if (!hisa_args_ok(k, B, keep) || !select_fits(keep, std::max(0, (hi.max_k + B - 1) / B - 2)))
+        return DSA_ERR_UNSUPPORTED;
     if ((s = check_tensors(b, Q, K, W)) != DSA_OK) return s;
     if (b->num_queries > 0 && (!idx || !pooled)) return DSA_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(pooled) & 15) return DSA_ERR_INVALID_ARG;
     HisaPlan p;
-    if ((s = check_ws(ws, ws_bytes, hisa_plan(nullptr, b, hi, B, keep, &p))) != DSA_OK) return s;
-    hisa_plan(static_cast<char*>(ws), b, hi, B, keep, &p);
+    if ((s = check_ws(ws, ws_bytes, hisa_plan(nullptr, b, hi, k, B, keep, &p))) != DSA_OK) return s;
+    hisa_plan(static_cast<char*>(ws), b, hi, k, B, keep, &p);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((s = clear_status(ws, st)) != DSA_OK) return s;
     const int32_t nq = b->num_queries;
@@ -802,7 +871,7 @@ dsa_status hisa_index(const dsa_batch* b, const void* Q, const void* K, const fl
     const std::vector<int32_t> qoff = iota_host(nq);
     const TcSource src{Q, nq, W, p.query_off, qoff.data(), nq};
     return tc_score_and_select(p.token_rows, nq, src, H, D, K, b->num_keys, b->k_offsets, m, (keep + 2) * B, p.S,
-                               p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, nullptr, st);
+                               p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, nullptr, st, p.split);
 }
 
 // ---------------------------------------------------------------- profiling
@@ -908,11 +977,12 @@ extern "C" dsa_status dsa_index_topk_static(const dsa_batch* b, const void* Q, c
     HostInfo hi;
     dsa_status s = check_batch(b, &hi);
     if (s != DSA_OK) return s;
-    if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
+    if (k < 1 || k > kMaxK || !select_fits(k, hi.max_k)) return DSA_ERR_UNSUPPORTED;
     DensePlan p;
-    if (dense_plan(nullptr, b, hi, false, &p) > kStaticScratchBytes) return DSA_ERR_WORKSPACE;
+    if (dense_plan(nullptr, b, hi, k, &p) > kStaticScratchBytes) return DSA_ERR_WORKSPACE;
     void* ws = nullptr;
     if ((s = static_scratch(&ws)) != DSA_OK) return s;
-    // dsa_index_topk clears the status word at the start of every call; nothing else must start at zero.
+    // dsa_index_topk clears the workspace header (status word, select counters) at the start of
+    // every call; nothing else must start at zero.
     return dsa_index_topk(b, Q, K, W, k, idx, scores, ws, kStaticScratchBytes, stream);
 }

@@ -227,10 +227,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int i = 0; i < nkt && !*abort_flag; ++i) {
                     if (!tc_wait(&full[stage], phase, a.status, 3, abort_flag)) break;
                     tc_fence_after();
-                    for (int acc = 0; acc < n_acc; ++acc) {
-                        if (!tc_wait(&tempty[acc], tph[acc] ^ 1u, a.status, 4, abort_flag)) break;
+                    for (int qb = 0; qb < n_acc; ++qb) {
+                        // one query block: the two accumulators alternate tile by tile
+                        const int slot = n_acc == 1 ? (i & 1) : qb;
+                        if (!tc_wait(&tempty[slot], tph[slot] ^ 1u, a.status, 4, abort_flag)) break;
                         tc_fence_after();
-                        const uint32_t d = tmem + acc * 256;
+                        const uint32_t d = tmem + slot * 256;
 #pragma unroll
                         for (int kk = 0; kk < SH::KSTEPS; ++kk) {
                             const int bx = kk / (SH::BOXC / 16);
@@ -238,11 +240,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             const uint64_t ad =
                                 smem_desc_kmajor(smem_u32(sK + stage * SH::KTILE + bx * SH::KBOX) + ko, SH::ROWB);
                             const uint64_t bd =
-                                smem_desc_kmajor(smem_u32(sQ + acc * SH::QACC + bx * SH::QBOX) + ko, SH::ROWB);
-                            tc_mma(d, ad, bd, idesc[acc], kk > 0 ? 1u : 0u);
+                                smem_desc_kmajor(smem_u32(sQ + qb * SH::QACC + bx * SH::QBOX) + ko, SH::ROWB);
+                            tc_mma(d, ad, bd, idesc[qb], kk > 0 ? 1u : 0u);
                         }
-                        tc_commit(&tfull[acc]);
-                        tph[acc] ^= 1u;
+                        tc_commit(&tfull[slot]);
+                        tph[slot] ^= 1u;
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == n_stages) { stage = 0; phase ^= 1u; }
@@ -260,12 +262,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t tph[2] = {0, 0};
         for (int i = 0; i < nkt; ++i) {
             const int key = (u.kt0 + i) * 128 + quarter * 32 + lane;
-            for (int acc = 0; acc < n_acc; ++acc) {
-                if (!tc_wait(&tfull[acc], tph[acc], a.status, 5, abort_flag)) break;
-                tph[acc] ^= 1u;
+            for (int acc = 0; acc < n_acc; ++acc) {   // acc: query block
+                const int slot = n_acc == 1 ? (i & 1) : acc;
+                if (!tc_wait(&tfull[slot], tph[slot], a.status, 5, abort_flag)) break;
+                tph[slot] ^= 1u;
                 tc_fence_after();
                 float v[128];
-                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + acc * 256 + half * 128;
+                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + slot * 256 + half * 128;
                 tmem_ld32(taddr, v);
                 tmem_ld32(taddr + 32, v + 32);
                 tmem_ld32(taddr + 64, v + 64);
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tmem_ld_wait();
                 tmem_regs_ready<128>(v);
                 tc_fence_before();
-                mbar_arrive(&tempty[acc]);   // the accumulator may be overwritten from here on
+                mbar_arrive(&tempty[slot]);   // the accumulator may be overwritten from here on
 
                 const int jbase = acc * NQA + half * QH;
 #pragma unroll

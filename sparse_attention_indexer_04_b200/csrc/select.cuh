@@ -4,28 +4,38 @@
 // largest key of the row) plus the lowest columns whose key equals T: ties
 // go to the lower key index.  Columns are written in ascending order.
 //
-// One CTA of 256 threads ranks one row, keeping little state so several rows
-// are in flight per SM:
-//   1. threshold: the keys of 2048 evenly spaced columns are ranked and the
-//      one at rank k*m/n plus a 4-sigma margin becomes tau (rows with at most
-//      select_buf_cap(k) columns skip this and keep every column);
+// A row is ranked in four steps:
+//   1. threshold: the keys of m evenly spaced columns (m = 2048 per 64K
+//      columns, at most 8192) are ranked and the one at rank k*m/n plus a
+//      4-sigma margin becomes tau (rows that fit the candidate buffer skip
+//      this and keep every column);
 //   2. one streaming pass appends every column with key >= tau to a
-//      shared-memory buffer (select_buf_cap(k) entries);
+//      candidate buffer (about 1.75 k entries);
 //   3. if at least k columns passed and none was dropped, the top k of the
 //      row are exactly the top k of the buffer: an 8-bit radix select over
 //      the buffer finds T and the number of T-ties to take.  Otherwise
 //      (a misleading sample) T is found by radix passes over the whole row;
 //   4. the selected columns are marked in two bitmaps (> T, == T) and emitted
 //      in column order, taking the first ties.
+// select_stream_kernel gives each row one CTA (many rows: prefill).
+// select_split_kernel gives each row several CTAs that share step 2 through
+// a global buffer, the last of them finishing the row (few long rows: decode).
 #pragma once
 
 #include "common.cuh"
 
 namespace dsa {
 
-constexpr int kSelThreads = 256;
-constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kSampleMax = 2048;
+constexpr int kSampleMin = 2048;
+constexpr int kSampleMax = 8192;
+
+// Sample size for a row of n columns: 2048 per 65536 columns, 2048 to 8192, so the expected rank of
+// the k-th largest key in the sample (k * m / n) stays at 64 or more up to n = 256K for k = 2048.
+__host__ __device__ inline int select_sample_size(int n)
+{
+    const int m = kSampleMin * ((n + 65535) / 65536);
+    return m < kSampleMin ? kSampleMin : (m > kSampleMax ? kSampleMax : m);
+}
 
 // Candidate buffer entries for top-k: at least 4096 and 1.75 k.
 __host__ __device__ inline int select_buf_cap(int k)
@@ -42,7 +52,8 @@ struct SelectArgs {
     const float* S;          // score row r at S + src_row * ld_s
     int64_t ld_s;
     int32_t src_from_list;   // 1: the score row is rows[r].list instead of r
-    int32_t buf_cap;         // candidate buffer entries (select_stream_kernel)
+    int32_t buf_cap;         // candidate buffer entries
+    int32_t sample_bytes;    // shared memory of the sample: select_sample_bytes(max_cols)
     int32_t* out_idx;        // [n_rows, ld_idx]
     int64_t ld_idx;
     float* out_score;        // nullable, [n_rows, ld_score]
@@ -50,11 +61,14 @@ struct SelectArgs {
 };
 
 
-// Dynamic shared memory of select_stream_kernel for rows of up to max_cols columns.
+// Dynamic shared memory of the select kernels for rows of up to max_cols columns: the sample, the
+// candidate buffer and two bitmaps of the row's columns.
+__host__ __device__ inline size_t select_sample_bytes(int max_cols) { return (size_t)select_sample_size(max_cols) * 4; }
+
 __host__ __device__ inline size_t select_smem_bytes(int max_cols, int buf_cap)
 {
     const size_t words = (size_t)(max_cols + 31) / 32;
-    return kSampleMax * 4 + (size_t)buf_cap * 8 + 2 * words * 4;
+    return select_sample_bytes(max_cols) + (size_t)buf_cap * 8 + 2 * words * 4;
 }
 
 // Exact rank selection among `count` keys given by get(i): returns the key T
@@ -125,129 +139,150 @@ __device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, 
     return lo + prefix;
 }
 
+// Shared scalars of one selection CTA.
 template <int NT>
-__global__ void __launch_bounds__(NT) select_stream_kernel(SelectArgs a)
+struct SelScalars {
+    uint32_t hist[256];
+    uint32_t scratch[2 * (NT / 32) + 2];
+    uint32_t count;   // candidates seen by the append pass
+    uint32_t base;    // split rows: this CTA's first slot in the row's global buffer
+    uint32_t last;    // split rows: this CTA finishes the row
+    uint32_t wgt[NT / 32], weq[NT / 32];
+};
+
+// 1. tau for a row of n > k columns: 0 (every column is a candidate) when n <= buf_cap, else
+// the key at rank expect + 4 sqrt(expect) + 4 among m = select_sample_size(n) evenly spaced
+// columns, expect = k * m / n (the expected rank of the k-th largest key in the sample, plus a
+// margin).
+template <int NT>
+__device__ __forceinline__ uint32_t sel_threshold(const float* src, int n, int k, int buf_cap, uint32_t* sample,
+                                                  SelScalars<NT>& sh)
 {
-    constexpr int kSelThreads = NT;
-    constexpr int kSelWarps = NT / 32;
-    extern __shared__ __align__(16) uint8_t sel_smem[];
-    uint32_t* sample = reinterpret_cast<uint32_t*>(sel_smem);
-    const int kBufCap = a.buf_cap;
-    uint64_t* buf = reinterpret_cast<uint64_t*>(sel_smem + kSampleMax * 4);
-    uint32_t* gtmap = reinterpret_cast<uint32_t*>(sel_smem + kSampleMax * 4 + (size_t)kBufCap * 8);
-    __shared__ uint32_t hist[256];
-    __shared__ uint32_t scratch[2 * kSelWarps + 2];
-    __shared__ uint32_t s_count;
-    __shared__ uint32_t s_wgt[kSelWarps], s_weq[kSelWarps];
+    if (n <= buf_cap) return 0u;
+    const int tid = threadIdx.x;
+    const int m = select_sample_size(n);   // a multiple of 2048
+    constexpr int J = kSampleMin / NT;     // sample loads in flight per thread
+    for (int j0 = 0; j0 < m; j0 += kSampleMin) {
+        float x[J];
+#pragma unroll
+        for (int j = 0; j < J; ++j) x[j] = __ldg(src + (int)(((int64_t)(j0 + tid + j * NT) * n) / m));
+#pragma unroll
+        for (int j = 0; j < J; ++j) sample[j0 + tid + j * NT] = score_key(x[j]);
+    }
+    const float expect = (float)k * m / n;
+    int rank = (int)ceilf(expect + 4.f * sqrtf(expect) + 4.f);
+    rank = min(rank, m);
+    __syncthreads();
+    return radix_select<NT>([&](int i) { return sample[i]; }, m, rank, sh.hist, sh.scratch);
+}
 
-    const int r = blockIdx.x;
-    const RowDesc rd = a.rows[r];
-    const int n = rd.ncols;
-    const int k = a.k;
-    const float* src = a.S + (int64_t)(a.src_from_list ? rd.list : r) * a.ld_s;
+// 2. Appends (key << 32 | column) of every column c in [c0, c1) whose key is >= tau to buf, one
+// shared atomic per warp and batch; sh.count (zero on entry) counts them all, entries past cap
+// are dropped.  c0 is a multiple of 4.
+template <int NT>
+__device__ __forceinline__ void sel_append(const float* src, int c0, int c1, uint32_t tau, uint64_t* buf, int cap,
+                                           SelScalars<NT>& sh)
+{
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nwords = (n + 31) >> 5;
-    uint32_t* eqmap = gtmap + nwords;
-    int32_t* oidx = a.out_idx + (int64_t)r * a.ld_idx;
-    float* osc = a.out_score ? a.out_score + (int64_t)r * a.ld_score : nullptr;
+    // nv: how many of x's four columns (c .. c+3) exist.
+    auto keep4 = [&](float4 x, int c, int nv) {
+        const uint32_t u0 = score_key(x.x), u1 = score_key(x.y), u2 = score_key(x.z), u3 = score_key(x.w);
+        const bool p0 = nv > 0 && u0 >= tau, p1 = nv > 1 && u1 >= tau, p2 = nv > 2 && u2 >= tau,
+                   p3 = nv > 3 && u3 >= tau;
+        const uint32_t b0 = __ballot_sync(0xffffffffu, p0), b1 = __ballot_sync(0xffffffffu, p1);
+        const uint32_t b2 = __ballot_sync(0xffffffffu, p2), b3 = __ballot_sync(0xffffffffu, p3);
+        const uint32_t total = __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3);
+        if (total == 0) return;
+        uint32_t slot = 0;
+        if (lane == 0) slot = atomicAdd(&sh.count, total);
+        slot = __shfl_sync(0xffffffffu, slot, 0);
+        const uint32_t lt = lanemask_lt();
+        uint32_t o = slot + __popc(b0 & lt);
+        if (p0 && o < (uint32_t)cap) buf[o] = ((uint64_t)u0 << 32) | (uint32_t)c;
+        o = slot + __popc(b0) + __popc(b1 & lt);
+        if (p1 && o < (uint32_t)cap) buf[o] = ((uint64_t)u1 << 32) | (uint32_t)(c + 1);
+        o = slot + __popc(b0) + __popc(b1) + __popc(b2 & lt);
+        if (p2 && o < (uint32_t)cap) buf[o] = ((uint64_t)u2 << 32) | (uint32_t)(c + 2);
+        o = slot + __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3 & lt);
+        if (p3 && o < (uint32_t)cap) buf[o] = ((uint64_t)u3 << 32) | (uint32_t)(c + 3);
+    };
+    const float* s = src + c0;
+    const int len = c1 - c0;
+    const bool vec = (reinterpret_cast<uintptr_t>(s) & 15) == 0;
+    const int n4 = vec ? (len >> 2) : 0;
+    const float4* s4 = reinterpret_cast<const float4*>(s);
+    constexpr int U = 8;   // 16-byte loads in flight per thread
+    for (int i4 = warp * 32; i4 < n4; i4 += U * NT) {   // warp-uniform trip count
+        float4 x[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i4 + u * NT + lane;
+            x[u] = i < n4 ? __ldg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i4 + u * NT + lane;
+            keep4(x[u], c0 + 4 * i, i < n4 ? 4 : 0);
+        }
+    }
+    for (int j0 = 4 * n4 + warp * 32; j0 < len; j0 += NT) {   // tail (or the whole range if unaligned)
+        const int j = j0 + lane;
+        const float v0 = j < len ? __ldg(s + j) : 0.f;
+        keep4(make_float4(v0, 0.f, 0.f, 0.f), c0 + j, j < len ? 1 : 0);
+    }
+}
 
-    for (int w = tid; w < 2 * nwords; w += kSelThreads) gtmap[w] = 0;
-    uint32_t thresh = 0;   // T: the k-th largest key (0 when every column is taken)
-    int krem = n;          // ties at T still to take
-    if (n > k) {
-        // ---- 1. threshold from a sample (or every column for short rows)
-        uint32_t tau = 0;
-        if (n > kBufCap) {
-            const int m = kSampleMax;
-            float x[kSampleMax / kSelThreads];   // all sample loads in flight at once
-#pragma unroll
-            for (int j = 0; j < kSampleMax / kSelThreads; ++j)
-                x[j] = __ldg(src + (int)(((int64_t)(tid + j * kSelThreads) * n) / m));
-#pragma unroll
-            for (int j = 0; j < kSampleMax / kSelThreads; ++j) sample[tid + j * kSelThreads] = score_key(x[j]);
-            const float expect = (float)k * m / n;
-            int rank = (int)ceilf(expect + 4.f * sqrtf(expect) + 4.f);
-            rank = min(rank, m);
-            __syncthreads();
-            tau = radix_select<NT>([&](int i) { return sample[i]; }, m, rank, hist, scratch);
-        }
-        // ---- 2. one pass: every column with key >= tau into the buffer
-        if (tid == 0) s_count = 0;
-        __syncthreads();
-        // Appends the columns of this lane that pass, one shared atomic per warp.
-        // nv: how many of x's four columns (c .. c+3) exist.
-        auto keep4 = [&](float4 x, int c, int nv) {
-            const uint32_t u0 = score_key(x.x), u1 = score_key(x.y), u2 = score_key(x.z), u3 = score_key(x.w);
-            const bool p0 = nv > 0 && u0 >= tau, p1 = nv > 1 && u1 >= tau, p2 = nv > 2 && u2 >= tau,
-                       p3 = nv > 3 && u3 >= tau;
-            const uint32_t b0 = __ballot_sync(0xffffffffu, p0), b1 = __ballot_sync(0xffffffffu, p1);
-            const uint32_t b2 = __ballot_sync(0xffffffffu, p2), b3 = __ballot_sync(0xffffffffu, p3);
-            const uint32_t total = __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3);
-            if (total == 0) return;
-            uint32_t slot = 0;
-            if (lane == 0) slot = atomicAdd(&s_count, total);
-            slot = __shfl_sync(0xffffffffu, slot, 0);
-            const uint32_t lt = lanemask_lt();
-            uint32_t o = slot + __popc(b0 & lt);
-            if (p0 && o < (uint32_t)kBufCap) buf[o] = ((uint64_t)u0 << 32) | (uint32_t)c;
-            o = slot + __popc(b0) + __popc(b1 & lt);
-            if (p1 && o < (uint32_t)kBufCap) buf[o] = ((uint64_t)u1 << 32) | (uint32_t)(c + 1);
-            o = slot + __popc(b0) + __popc(b1) + __popc(b2 & lt);
-            if (p2 && o < (uint32_t)kBufCap) buf[o] = ((uint64_t)u2 << 32) | (uint32_t)(c + 2);
-            o = slot + __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3 & lt);
-            if (p3 && o < (uint32_t)kBufCap) buf[o] = ((uint64_t)u3 << 32) | (uint32_t)(c + 3);
-        };
-        const bool vec = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
-        const int n4 = vec ? (n >> 2) : 0;
-        const float4* s4 = reinterpret_cast<const float4*>(src);
-        constexpr int U = 8;   // 16-byte loads in flight per thread
-        for (int c4 = warp * 32; c4 < n4; c4 += U * kSelThreads) {   // warp-uniform trip count
-            float4 x[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int i = c4 + u * kSelThreads + lane;
-                x[u] = i < n4 ? __ldg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int i = c4 + u * kSelThreads + lane;
-                keep4(x[u], 4 * i, i < n4 ? 4 : 0);
-            }
-        }
-        for (int c0 = 4 * n4 + warp * 32; c0 < n; c0 += kSelThreads) {   // tail (or the whole row if unaligned)
-            const int c = c0 + lane;
-            const float v0 = c < n ? __ldg(src + c) : 0.f;
-            keep4(make_float4(v0, 0.f, 0.f, 0.f), c, c < n ? 1 : 0);
-        }
-        __syncthreads();
-        const int count = (int)s_count;
-        krem = k;
-        if (count >= k && count <= kBufCap) {
-            // ---- 3. exact top-k of the buffer
-            thresh = radix_select<NT>([&](int i) { return (uint32_t)(buf[i] >> 32); }, count, krem, hist, scratch);
-            for (int i = tid; i < count; i += kSelThreads) {
-                const uint32_t u = (uint32_t)(buf[i] >> 32), c = (uint32_t)buf[i];
-                if (u > thresh) atomicOr(&gtmap[c >> 5], 1u << (c & 31));
-                else if (u == thresh) atomicOr(&eqmap[c >> 5], 1u << (c & 31));
-            }
-        } else {
-            // ---- 3'. the sample misled: exact selection over the whole row
-            thresh = radix_select<NT>([&](int i) { return score_key(__ldg(src + i)); }, n, krem, hist, scratch);
-            for (int c = tid; c < n; c += kSelThreads) {
-                const uint32_t u = score_key(__ldg(src + c));
-                if (u > thresh) atomicOr(&gtmap[c >> 5], 1u << (c & 31));
-                else if (u == thresh) atomicOr(&eqmap[c >> 5], 1u << (c & 31));
-            }
+// 3. Marks the row's top k in the bitmaps (> T in gtmap, == T in eqmap, both zeroed) and returns
+// in krem how many ties at T to take.  From the candidate buffer when it holds every column
+// with key >= tau (k <= count <= cap), else (a misleading sample) by radix passes over the
+// whole row.
+template <int NT>
+__device__ __forceinline__ void sel_mark(const float* src, int n, int k, const uint64_t* buf, int count, int cap,
+                                         int& krem, uint32_t* gtmap, uint32_t* eqmap, SelScalars<NT>& sh)
+{
+    const int tid = threadIdx.x;
+    krem = k;
+    if (count >= k && count <= cap) {
+        const uint32_t thresh =
+            radix_select<NT>([&](int i) { return (uint32_t)(buf[i] >> 32); }, count, krem, sh.hist, sh.scratch);
+        for (int i = tid; i < count; i += NT) {
+            const uint32_t u = (uint32_t)(buf[i] >> 32), c = (uint32_t)buf[i];
+            if (u > thresh) atomicOr(&gtmap[c >> 5], 1u << (c & 31));
+            else if (u == thresh) atomicOr(&eqmap[c >> 5], 1u << (c & 31));
         }
     } else {
-        __syncthreads();
-        for (int w = tid; w < nwords; w += kSelThreads)
-            gtmap[w] = (w + 1) * 32 <= n ? 0xffffffffu : ((1u << (n & 31)) - 1u);
+        const uint32_t thresh =
+            radix_select<NT>([&](int i) { return score_key(__ldg(src + i)); }, n, krem, sh.hist, sh.scratch);
+        for (int c = tid; c < n; c += NT) {
+            const uint32_t u = score_key(__ldg(src + c));
+            if (u > thresh) atomicOr(&gtmap[c >> 5], 1u << (c & 31));
+            else if (u == thresh) atomicOr(&eqmap[c >> 5], 1u << (c & 31));
+        }
     }
-    __syncthreads();
+}
 
-    // ---- 4. emit in column order: warp w owns words [w*wpw, (w+1)*wpw)
-    const int wpw = (nwords + kSelWarps - 1) / kSelWarps;
+// Rows of at most k columns: every column is taken.
+template <int NT>
+__device__ __forceinline__ void sel_mark_all(int n, uint32_t* gtmap)
+{
+    const int nwords = (n + 31) >> 5;
+    for (int w = threadIdx.x; w < nwords; w += NT)
+        gtmap[w] = (w + 1) * 32 <= n ? 0xffffffffu : ((1u << (n & 31)) - 1u);
+}
+
+// 4. Emits the marked columns in column order (all of gtmap, the first krem of eqmap), then pads
+// the row to k with -1 (and NaN scores).  Warp w owns bitmap words [w*wpw, (w+1)*wpw).
+template <int NT>
+__device__ __forceinline__ void sel_emit(const SelectArgs& a, const RowDesc& rd, int r, const float* src, int n,
+                                         int krem, const uint32_t* gtmap, const uint32_t* eqmap, SelScalars<NT>& sh)
+{
+    constexpr int kWarps = NT / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int k = a.k;
+    const int nwords = (n + 31) >> 5;
+    int32_t* oidx = a.out_idx + (int64_t)r * a.ld_idx;
+    float* osc = a.out_score ? a.out_score + (int64_t)r * a.ld_score : nullptr;
+    const int wpw = (nwords + kWarps - 1) / kWarps;
     const int w0 = warp * wpw, w1 = min(w0 + wpw, nwords);
     uint32_t gt = 0, eq = 0;
     for (int w = w0 + lane; w < w1; w += 32) { gt += __popc(gtmap[w]); eq += __popc(eqmap[w]); }
@@ -256,10 +291,10 @@ __global__ void __launch_bounds__(NT) select_stream_kernel(SelectArgs a)
         gt += __shfl_xor_sync(0xffffffffu, gt, o);
         eq += __shfl_xor_sync(0xffffffffu, eq, o);
     }
-    if (lane == 0) { s_wgt[warp] = gt; s_weq[warp] = eq; }
+    if (lane == 0) { sh.wgt[warp] = gt; sh.weq[warp] = eq; }
     __syncthreads();
     uint32_t eq_rank = 0, out = 0;
-    for (int w = 0; w < warp; ++w) { out += s_wgt[w]; eq_rank += s_weq[w]; }
+    for (int w = 0; w < warp; ++w) { out += sh.wgt[w]; eq_rank += sh.weq[w]; }
     out += min(eq_rank, (uint32_t)krem);
     for (int wb = w0; wb < w1; wb += 32) {
         const int w = wb + lane;
@@ -294,10 +329,115 @@ __global__ void __launch_bounds__(NT) select_stream_kernel(SelectArgs a)
         eq_rank += __shfl_sync(0xffffffffu, pre_e, 31);
     }
     const int n_out = min(n, k);
-    for (int j = n_out + tid; j < k; j += kSelThreads) {
+    for (int j = n_out + tid; j < k; j += NT) {
         oidx[j] = -1;
         if (osc) osc[j] = __int_as_float(0x7fc00000);
     }
+}
+
+// One CTA per row: steps 1-4 above.
+template <int NT>
+__global__ void __launch_bounds__(NT) select_stream_kernel(SelectArgs a)
+{
+    extern __shared__ __align__(16) uint8_t sel_smem[];
+    uint32_t* sample = reinterpret_cast<uint32_t*>(sel_smem);
+    const int cap = a.buf_cap;
+    uint64_t* buf = reinterpret_cast<uint64_t*>(sel_smem + a.sample_bytes);
+    uint32_t* gtmap = reinterpret_cast<uint32_t*>(sel_smem + a.sample_bytes + (size_t)cap * 8);
+    __shared__ SelScalars<NT> sh;
+
+    const int r = blockIdx.x;
+    const RowDesc rd = a.rows[r];
+    const int n = rd.ncols;
+    const int k = a.k;
+    const float* src = a.S + (int64_t)(a.src_from_list ? rd.list : r) * a.ld_s;
+    const int nwords = (n + 31) >> 5;
+    uint32_t* eqmap = gtmap + nwords;
+
+    for (int w = threadIdx.x; w < 2 * nwords; w += NT) gtmap[w] = 0;
+    int krem = n;   // ties at T still to take (every column when n <= k)
+    if (n > k) {
+        const uint32_t tau = sel_threshold<NT>(src, n, k, cap, sample, sh);
+        if (threadIdx.x == 0) sh.count = 0;
+        __syncthreads();
+        sel_append<NT>(src, 0, n, tau, buf, cap, sh);
+        __syncthreads();
+        sel_mark<NT>(src, n, k, buf, (int)sh.count, cap, krem, gtmap, eqmap, sh);
+    } else {
+        __syncthreads();
+        sel_mark_all<NT>(n, gtmap);
+    }
+    __syncthreads();
+    sel_emit<NT>(a, rd, r, src, n, krem, gtmap, eqmap, sh);
+}
+
+// Few long rows: P CTAs per row (blockIdx.x = r * P + p).  Every CTA of a row derives the same
+// tau from the row's sample (step 1) and appends the candidates of its column chunk (step 2)
+// to the row's global buffer gbuf[r * cap, (r + 1) * cap), counting them in ctr[2r]; the last
+// CTA of the row to finish (ticket ctr[2r + 1]) ranks the buffer and writes the row (steps
+// 3-4), then zeroes the row's two counters.  ctr must be zero at launch.
+template <int NT>
+__global__ void __launch_bounds__(NT) select_split_kernel(SelectArgs a, uint64_t* gbuf, uint32_t* ctr, int P)
+{
+    extern __shared__ __align__(16) uint8_t sel_smem[];
+    uint32_t* sample = reinterpret_cast<uint32_t*>(sel_smem);
+    const int cap = a.buf_cap;
+    uint64_t* buf = reinterpret_cast<uint64_t*>(sel_smem + a.sample_bytes);
+    uint32_t* gtmap = reinterpret_cast<uint32_t*>(sel_smem + a.sample_bytes + (size_t)cap * 8);
+    __shared__ SelScalars<NT> sh;
+
+    const int r = blockIdx.x / P, p = blockIdx.x % P;
+    const RowDesc rd = a.rows[r];
+    const int n = rd.ncols;
+    const int k = a.k;
+    const float* src = a.S + (int64_t)(a.src_from_list ? rd.list : r) * a.ld_s;
+    const int tid = threadIdx.x;
+    uint64_t* g = gbuf + (int64_t)r * cap;
+
+    if (n > k) {
+        const uint32_t tau = sel_threshold<NT>(src, n, k, cap, sample, sh);
+        const int chunk = ((n + P - 1) / P + 127) & ~127;
+        const int c0 = min(n, p * chunk), c1 = min(n, c0 + chunk);
+        if (tid == 0) sh.count = 0;
+        __syncthreads();
+        sel_append<NT>(src, c0, c1, tau, buf, cap, sh);
+        __syncthreads();
+        // the whole count goes into the row's total, so a chunk that overflowed its own buffer
+        // also overflows the row's
+        if (tid == 0) sh.base = sh.count > 0 ? atomicAdd(&ctr[2 * r], sh.count) : 0u;
+        __syncthreads();
+        const uint32_t base = sh.base, local = min(sh.count, (uint32_t)cap);
+        for (uint32_t i = tid; i < local && base + i < (uint32_t)cap; i += NT) g[base + i] = buf[i];
+        __threadfence();
+    }
+    __syncthreads();
+    if (tid == 0) sh.last = atomicAdd(&ctr[2 * r + 1], 1u) == (uint32_t)(P - 1) ? 1u : 0u;
+    __syncthreads();
+    if (!sh.last) return;
+
+    // ---- the row's last CTA: every other CTA's candidates are in g
+    __threadfence();
+    const int nwords = (n + 31) >> 5;
+    uint32_t* eqmap = gtmap + nwords;
+    for (int w = tid; w < 2 * nwords; w += NT) gtmap[w] = 0;
+    if (tid == 0) {
+        sh.count = *reinterpret_cast<volatile uint32_t*>(&ctr[2 * r]);
+        ctr[2 * r] = 0u;       // ready for the next launch
+        ctr[2 * r + 1] = 0u;
+    }
+    __syncthreads();
+    int krem = n;
+    if (n > k) {
+        const int count = (int)sh.count;
+        if (count >= k && count <= cap)
+            for (int i = tid; i < count; i += NT) buf[i] = __ldcg(reinterpret_cast<const unsigned long long*>(g) + i);
+        __syncthreads();
+        sel_mark<NT>(src, n, k, buf, count, cap, krem, gtmap, eqmap, sh);
+    } else {
+        sel_mark_all<NT>(n, gtmap);
+    }
+    __syncthreads();
+    sel_emit<NT>(a, rd, r, src, n, krem, gtmap, eqmap, sh);
 }
 
 }  // namespace dsa

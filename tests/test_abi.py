@@ -96,6 +96,8 @@ def test_argument_errors_return_before_any_launch():
     assert call_topk(bad) == 1
     lib = dsa.library()
     assert lib.dsa_index_topk(None, None, None, None, 4, None, None, None, 0, None) == 1
+    # a row too long for the selection's shared memory (two column bitmaps) is refused up front
+    assert call_topk(host_layout([1], [1_000_000]), k=2048) == 2
 
 
 def test_pivot_and_hisa_argument_errors():

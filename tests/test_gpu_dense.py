@@ -119,14 +119,16 @@ def test_full_size_prefill_32k_sampled_rows():
     assert np.all(idx.max(1) <= np.arange(b.n_q))
 
 
+@pytest.mark.parametrize("n_rows", [2, 300])
 @pytest.mark.parametrize("sampled_high", [True, False])
-def test_select_when_the_even_sample_misleads(sampled_high):
+def test_select_when_the_even_sample_misleads(sampled_high, n_rows):
     """The top-k picks a threshold from 2048 evenly spaced columns of a long row.  Keys that make exactly
     those columns score high (too few columns then pass the threshold) or low (too many pass) must still
-    give the exact answer: integer inputs, compared exactly with the oracle."""
+    give the exact answer: integer inputs, compared exactly with the oracle.  Two rows take the split
+    select (several CTAs per row), 300 rows the one-CTA-per-row select."""
     L, k = 20000, 3000
-    b = workloads.ragged(30, [2], [L], H=1, d=32, k=k, integer=True)
-    sampled = np.unique((np.arange(2048, dtype=np.int64) * (L - 1 + 1)) // 2048)    # n = L for the last query
+    b = workloads.ragged(30, [n_rows], [L], H=1, d=32, k=k, integer=True)
+    sampled = np.unique((np.arange(2048, dtype=np.int64) * L) // 2048)    # the sample of a row of n = L
     hi, lo = (3.0, 1.0) if sampled_high else (1.0, 3.0)
     K = np.full((L, 32), lo, np.float32)
     K[sampled] = hi
@@ -134,5 +136,19 @@ def test_select_when_the_even_sample_misleads(sampled_high):
     b.K = torch.as_tensor(K).to(torch.bfloat16)
     b.Q = torch.ones_like(b.Q)
     b.W = torch.ones_like(b.W)
-    b.q_pos = torch.tensor([L - 2, L - 1], dtype=torch.int32)
+    pos = np.full(n_rows, L - 1, np.int32)
+    pos[0] = L - 2
+    b.q_pos = torch.as_tensor(pos)
     exact_topk(b, k)
+
+
+@pytest.mark.parametrize("seed,q_lens,k_lens,k,mode", [
+    (40, [2, 1, 3], [9000, 20000, 4500], 1000, "suffix"),
+    (41, [2, 2], [30000, 700], 2048, "random"),
+    (42, [1] * 20, [5000 + 997 * i for i in range(20)], 512, "suffix"),
+])
+def test_few_long_rows_exact(seed, q_lens, k_lens, k, mode):
+    """Few rows of many columns (decode): each row is ranked by several CTAs that share one candidate
+    buffer.  Integer inputs (many ties across the CTAs' column chunks), a row shorter than k, clamped
+    positions; exact against the oracle."""
+    exact_topk(workloads.ragged(seed, q_lens, k_lens, H=4, d=32, k=k, integer=True, pos_mode=mode), k)
