@@ -94,6 +94,31 @@ dsa_status launched()
     return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
+// Launches a kernel, with programmatic stream serialization when `pdl`: it may then be
+// scheduled while the previous kernel on the stream still runs, and must call grid_dep_wait()
+// before it touches memory an earlier kernel writes or reads.
+template <typename... KArgs, typename... Args>
+void launch_pdl(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                Args... args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    (void)cudaLaunchKernelEx(&cfg, kern, args...);   // errors surface through launched()
+}
+
+// Programmatic launch pays off for the short kernels of decode (it hides each launch's latency
+// behind the previous kernel) and cost the multi-wave prefill kernels ~4% when measured, so it
+// is used when the grids involved fit in about two waves.
+bool latency_bound(int64_t ctas) { return ctas <= 2 * 148; }
+
 // ------------------------------------------------------------- profiling
 // Kernel kinds timed by the optional profiler (dsa_profile_*).
 enum ProfKind : int32_t {
@@ -236,17 +261,18 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
     const int P = select_parts(n_rows, max_cols);
     if (sp.buf && sp.ctr && n_rows <= sp.max_rows && P > 1) {
         if ((s = set_smem(select_split_kernel<512>, smem)) != DSA_OK) return s;
-        DSA_LAUNCH(kProfSelect, st, select_split_kernel<512><<<n_rows * P, 512, smem, st>>>(a, sp.buf, sp.ctr, P));
+        DSA_LAUNCH(kProfSelect, st, launch_pdl(true, select_split_kernel<512>, n_rows * P, 512, smem, st, a, sp.buf,
+                                               sp.ctr, P));
         return launched();
     }
     switch (select_threads(n_rows)) {
     case 512:
         if ((s = set_smem(select_stream_kernel<512>, smem)) != DSA_OK) return s;
-        DSA_LAUNCH(kProfSelect, st, select_stream_kernel<512><<<n_rows, 512, smem, st>>>(a));
+        DSA_LAUNCH(kProfSelect, st, launch_pdl(latency_bound(n_rows), select_stream_kernel<512>, n_rows, 512, smem, st, a));
         break;
     default:
         if ((s = set_smem(select_stream_kernel<256>, smem)) != DSA_OK) return s;
-        DSA_LAUNCH(kProfSelect, st, select_stream_kernel<256><<<n_rows, 256, smem, st>>>(a));
+        DSA_LAUNCH(kProfSelect, st, launch_pdl(latency_bound(n_rows), select_stream_kernel<256>, n_rows, 256, smem, st, a));
         break;
     }
     return launched();
@@ -380,7 +406,8 @@ dsa_status launch_tc_shape(const CUtensorMap& mq, const CUtensorMap& mk, const C
     const int smem = std::max((int)SH::smem_bytes(n_acc, stages), 120 * 1024);
     if (cudaFuncSetAttribute(score_tc_kernel<D, H>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return DSA_ERR_CUDA;
-    DSA_LAUNCH(kProfScoreTc, st, score_tc_kernel<D, H><<<n_units, kTcThreads, smem, st>>>(mq, mk, mkg, args));
+    DSA_LAUNCH(kProfScoreTc, st, launch_pdl(latency_bound(n_units), score_tc_kernel<D, H>, n_units, kTcThreads, smem, st,
+                                            mq, mk, mkg, args));
     return launched();
 }
 
@@ -404,7 +431,7 @@ dsa_status launch_tc_d(int H, const CUtensorMap& mq, const CUtensorMap& mk, cons
 // map(c) of the row's sequence.
 dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const TcSource& src, int H, int D,
                     const void* K, int64_t n_k, const int32_t* k_base, const ColMap& map, int32_t max_cols, float* S,
-                    int64_t ld, TcUnitOut* units, int32_t* tile_base, uint32_t* status, cudaStream_t st)
+                    int64_t ld, TcUnit* units, int32_t* tile_base, uint32_t* status, cudaStream_t st)
 {
     if (n_rows <= 0 || max_cols <= 0 || n_k <= 0) return DSA_OK;
     const int32_t TQ = tc_tile_rows(H);
@@ -416,20 +443,20 @@ dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const
     if (!make_tile_map(&mq, src.Q, src.q_rows * H, D, 256) || !make_tile_map(&mk, K, n_k, D, 128) ||
         !make_tile_map(&mkg, K, n_k, D, 1))
         return DSA_ERR_CUDA;
-    DSA_LAUNCH(kProfSetup, st, tc_units_kernel<<<1, 1024, 0, st>>>(rows, n_rows, row_base, src.seq_off, src.n_seqs,
-                                                                    TQ, splits, tile_base, units));
+    DSA_LAUNCH(kProfSetup, st, launch_pdl(latency_bound(int64_t(tiles) * splits), tc_units_kernel, 1, 1024, 0, st, rows,
+                                          n_rows, row_base, src.seq_off, src.n_seqs, TQ, splits, k_base, tile_base,
+                                          units));
     dsa_status s = launched();
     if (s != DSA_OK) return s;
     int32_t max_q = 0;
     for (int b = 0; b < src.n_seqs; ++b) max_q = std::max(max_q, src.seq_off_host[b + 1] - src.seq_off_host[b]);
     const int n_acc = std::min(max_q, TQ) > TQ / 2 ? 2 : 1;
     TcArgs a{};
-    a.units = reinterpret_cast<const TcUnit*>(units);
+    a.units = units;
     a.rows = rows;
     a.map = map;
     a.gather = gather ? 1 : 0;
     a.W = src.W;
-    a.k_base = k_base;
     a.S = S;
     a.ld_s = ld;
     a.status = status;
@@ -443,7 +470,7 @@ dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const
 // Tensor-core scoring then exact top-k, in row chunks that fit the score buffer.
 dsa_status tc_score_and_select(const RowDesc* rows, int32_t n_rows, const TcSource& src, int H, int D, const void* K,
                                int64_t n_k, const int32_t* k_base, const ColMap& map, int32_t max_cols, float* Sbuf,
-                               TcUnitOut* units, int32_t* tile_base, uint32_t* status, int32_t k, int32_t* idx,
+                               TcUnit* units, int32_t* tile_base, uint32_t* status, int32_t k, int32_t* idx,
                                int64_t ld_idx, float* scores, cudaStream_t st, const SelectSplit& sp = SelectSplit{})
 {
     const int64_t ld = score_ld(max_cols);
@@ -473,7 +500,7 @@ ColMap identity_map(int32_t offset = 0)
 struct DensePlan {
     RowDesc* rows;
     float* S;
-    TcUnitOut* units;
+    TcUnit* units;
     int32_t* tile_base;
     SelectSplit split;
 };
@@ -487,7 +514,7 @@ size_t dense_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k,
     const int64_t ld = score_ld(hi.max_k);
     const int32_t chunk = k == 0 ? nq : chunk_rows(nq, ld);
     const TcSource src{nullptr, 0, nullptr, nullptr, b->q_offsets_host, b->num_seqs};
-    p->units = c.take<TcUnitOut>(tc_unit_capacity(src, b->num_queries, chunk, b->num_heads, hi.max_k));
+    p->units = c.take<TcUnit>(tc_unit_capacity(src, b->num_queries, chunk, b->num_heads, hi.max_k));
     p->tile_base = c.take<int32_t>(b->num_seqs + 1);
     p->split = SelectSplit{};
     if (k > 0) {
@@ -509,7 +536,7 @@ struct PivotPlan {
     int32_t* cand;
     float* cand_score;
     float* S;
-    TcUnitOut* units;
+    TcUnit* units;
     int32_t* tile_base;
     int32_t* group_rows;   // [n_groups + 1] first query row of each group
 };
@@ -565,7 +592,7 @@ size_t pivot_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t G,
     const int32_t cap = std::max(tc_unit_capacity(src, count_groups(b, G), chunk_scan, b->num_heads, hi.max_k),
                                  tc_unit_capacity(srf, b->num_queries, chunk_rows(std::max(1, b->num_queries), ld_ref),
                                                   b->num_heads, C));
-    p->units = c.take<TcUnitOut>(cap);
+    p->units = c.take<TcUnit>(cap);
     p->tile_base = c.take<int32_t>(std::max(b->num_seqs, ng) + 1);
     p->group_rows = c.take<int32_t>(ng + 1);
     return c.off;
@@ -579,7 +606,7 @@ struct HisaPlan {
     int32_t* kept;
     float* S;
     int32_t* query_off;    // [n_q + 1] 0..n_q: every query is its own segment
-    TcUnitOut* units;
+    TcUnit* units;
     int32_t* tile_base;
     SelectSplit split;     // the token stage's select
 };
@@ -608,7 +635,7 @@ size_t hisa_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, 
     p->query_off = c.take<int32_t>(nq + 1);
     const std::vector<int32_t> qoff = iota_host(b->num_queries);
     const TcSource src{nullptr, 0, nullptr, nullptr, qoff.data(), b->num_queries};
-    p->units = c.take<TcUnitOut>(tc_unit_capacity(src, b->num_queries, chunk_rows(nq, ld_tok), b->num_heads,
+    p->units = c.take<TcUnit>(tc_unit_capacity(src, b->num_queries, chunk_rows(nq, ld_tok), b->num_heads,
                                                   (keep + 2) * B));
     p->tile_base = c.take<int32_t>(nq + 1);
     p->split = SelectSplit{};

@@ -92,6 +92,26 @@ __device__ __forceinline__ int32_t find_seq(const int32_t* offsets, int32_t n_se
     return lo;
 }
 
+// One work unit of the tensor-core scoring kernel: consecutive query rows of one segment and a
+// range of its key tiles, with what the TMA producer needs to start at once.
+struct TcUnit {
+    int32_t row0;    // first row of the unit in the launch's row array
+    int32_t nrows;   // consecutive rows of one segment
+    int32_t kt0;     // key tiles [kt0, kt1) of 128 keys, segment-local
+    int32_t kt1;
+    int32_t qrow;    // query row (Q / W) of row0
+    int32_t krow0;   // key row of the segment's key 0: k_base[seq]
+    int32_t pad_[2];
+};
+
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization may
+// start while its predecessor still runs; grid_dep_wait() returns once the predecessor grid has
+// completed and its memory is visible (at once for a kernel launched without it), and
+// grid_dep_launch() lets the successor's CTAs be scheduled once every CTA of this grid has
+// called it or exited.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t lanemask_lt()
 {
     uint32_t m;

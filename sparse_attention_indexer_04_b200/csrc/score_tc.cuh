@@ -35,13 +35,6 @@ constexpr int kTcThreads = 320;
 constexpr int kTcMaxStages = 8;
 constexpr uint32_t kErrSmemAlign = 3;
 
-struct TcUnit {
-    int32_t row0;    // first row of the unit in the launch's row array
-    int32_t nrows;   // consecutive queries of one sequence
-    int32_t kt0;     // key tiles [kt0, kt1) of 128 keys, sequence-local
-    int32_t kt1;
-};
-
 struct TcArgs {
     const TcUnit* units;
     const RowDesc* rows;
@@ -50,7 +43,6 @@ struct TcArgs {
     int32_t gather;          // 0: contiguous tiles, 1: gathered rows
     int32_t pad2_;
     const float* W;          // row rd.qrow: [H]
-    const int32_t* k_base;   // key row of (seq, key) = k_base[seq] + key
     float* S;                // score of launch row r, key s at S[r * ld_s + s]
     int64_t ld_s;
     uint32_t* status;
@@ -73,11 +65,20 @@ struct TcShape {
     static constexpr uint32_t NC_BYTES = 2u * NQA * 4;
     static constexpr uint32_t BAR_BYTES = 256;
 
+    // Q tiles, key stages, W, eligible counts; the barriers and TMEM slot sit in the last
+    // BAR_BYTES of the allocation, a place the prologue knows before the unit is read.
     __host__ __device__ static uint32_t smem_bytes(int n_acc, int n_stages)
     {
         return n_acc * QACC + n_stages * KTILE + W_BYTES + NC_BYTES + BAR_BYTES;
     }
 };
+
+__device__ __forceinline__ uint32_t dynamic_smem_size()
+{
+    uint32_t x;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(x));
+    return x;
+}
 
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, uint32_t* status, uint32_t where,
                                         volatile int32_t* abort_flag)
@@ -107,19 +108,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int QH = NQA / 2;   // queries of one accumulator handled by one epilogue half
 
     extern __shared__ __align__(1024) uint8_t smem[];
-    const TcUnit u = a.units[blockIdx.x];
-    if (u.kt1 <= u.kt0 || u.nrows <= 0) return;   // nothing to score (uniform exit)
-    if (smem_u32(smem) & 1023u) {                 // the swizzled tiles need 1024-byte alignment
+    if (smem_u32(smem) & 1023u) {   // the swizzled tiles need 1024-byte alignment (uniform exit)
         if (threadIdx.x == 0) record_error(a.status, kErrSmemAlign, blockIdx.x);
         return;
     }
-    const int n_acc = u.nrows > NQA ? 2 : 1;
     const int n_stages = a.n_stages;
-    uint8_t* sQ = smem;
-    uint8_t* sK = smem + n_acc * SH::QACC;
-    float* sW = reinterpret_cast<float*>(sK + n_stages * SH::KTILE);
-    int32_t* sNc = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(sW) + SH::W_BYTES);
-    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sNc) + SH::NC_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + dynamic_smem_size() - SH::BAR_BYTES);
     uint64_t* empty = full + n_stages;
     uint64_t* qfull = empty + n_stages;
     uint64_t* tfull = qfull + 1;
@@ -128,6 +122,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
 
+    // Prologue (may overlap the previous kernel): barriers, TMEM, descriptor prefetch.
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < n_stages; ++i) {
@@ -143,36 +138,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 1) tmem_alloc(tmem_slot, 512);
-    if (warp >= 2) {   // stage the tile's head weights and eligible counts
-        for (int i = threadIdx.x - 64; i < 2 * NQA * H; i += kTcThreads - 64) {
-            const int j = i / H;
-            sW[i] = j < u.nrows ? a.W[(int64_t)a.rows[u.row0 + j].qrow * H + (i % H)] : 0.f;
-        }
-        for (int j = threadIdx.x - 64; j < 2 * NQA; j += kTcThreads - 64)
-            sNc[j] = j < u.nrows ? a.rows[u.row0 + j].ncols : 0;
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(a.gather ? &tmKg : &tmK);
     }
+    if (warp == 1) tmem_alloc(tmem_slot, 512);
+    grid_dep_wait();     // the unit table and rows come from earlier kernels
+    // (no early launch of the next kernel: its CTAs waiting on freed SMs slowed decode down)
+    const TcUnit u = a.units[blockIdx.x];
+    const bool active = u.kt1 > u.kt0 && u.nrows > 0;   // uniform over the CTA
+    const int n_acc = u.nrows > NQA ? 2 : 1;
+    uint8_t* sQ = smem;
+    uint8_t* sK = sQ + n_acc * SH::QACC;
+    float* sW = reinterpret_cast<float*>(sK + n_stages * SH::KTILE);
+    int32_t* sNc = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(sW) + SH::W_BYTES);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const RowDesc first = a.rows[u.row0];
     const int nkt = u.kt1 - u.kt0;
 
-    if (warp == 0) {
+    if (!active) {
+        // nothing to score: fall through to the TMEM release
+    } else if (warp == 0) {
         // ------------------------------------------------------ TMA producer
-        const int krow0 = a.k_base[first.seq];
+        const int krow0 = u.krow0;
         if (lane == 0) {
-            prefetch_tensormap(&tmQ);
-            prefetch_tensormap(a.gather ? &tmKg : &tmK);
             mbar_arrive_expect_tx(qfull, n_acc * SH::QACC);
             for (int acc = 0; acc < n_acc; ++acc)
                 for (int bx = 0; bx < SH::NBOX; ++bx)
-                    tma_load_2d(sQ + acc * SH::QACC + bx * SH::QBOX, &tmQ, bx * SH::BOXC, (first.qrow + acc * NQA) * H,
+                    tma_load_2d(sQ + acc * SH::QACC + bx * SH::QBOX, &tmQ, bx * SH::BOXC, (u.qrow + acc * NQA) * H,
                                 qfull);
         }
-        int ncmax = 0;   // columns of the unit that exist (tiles past it read column 0's key)
-        for (int j = 0; j < u.nrows; ++j) ncmax = max(ncmax, sNc[j]);
+        // Gathered tiles: the columns of the unit that exist (tiles past them read column 0's key).
+        int ncmax = 0, list = 0;
+        if (a.gather) {
+            list = a.rows[u.row0].list;
+            for (int j = lane; j < u.nrows; j += 32) ncmax = max(ncmax, a.rows[u.row0 + j].ncols);
+            ncmax = __reduce_max_sync(0xffffffffu, ncmax);
+        }
+        const RowDesc first{0, 0, 0, list};   // map_col reads only the list row
         int stage = 0;
         uint32_t phase = 0;
         int issued = 0;
@@ -257,6 +262,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------------- epilogue
+        // the tile's head weights and eligible counts, shared by the 8 epilogue warps
+        for (int i = threadIdx.x - 64; i < 2 * NQA * H; i += kTcThreads - 64) {
+            const int j = i / H;
+            sW[i] = j < u.nrows ? a.W[(int64_t)a.rows[u.row0 + j].qrow * H + (i % H)] : 0.f;
+        }
+        for (int j = threadIdx.x - 64; j < 2 * NQA; j += kTcThreads - 64)
+            sNc[j] = j < u.nrows ? a.rows[u.row0 + j].ncols : 0;
+        asm volatile("bar.sync 1, 256;" ::: "memory");   // named barrier of the epilogue warps only
         const int quarter = warp & 3;           // TMEM lanes this warp may read
         const int half = (warp - 2) >> 2;       // which 128 columns of an accumulator
         uint32_t tph[2] = {0, 0};

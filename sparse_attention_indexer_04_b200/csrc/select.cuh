@@ -75,9 +75,12 @@ __host__ __device__ inline size_t select_smem_bytes(int max_cols, int buf_cap)
 // holding rank `krem` (1 = largest) and, in krem, how many keys equal to T
 // that rank reaches.  Digits are taken from (key - min), starting at the
 // highest bit where min and max differ, 8 bits at a time, so even the first
-// pass spreads the keys over many bins.  All threads call it.
+// pass spreads the keys over many bins.  With stop_bits > 0 only the top
+// stop_bits bits of (key - min) are resolved and the lower edge of that bin
+// is returned: a key <= T (krem is then meaningless).  All threads call it.
 template <int NT, typename Get>
-__device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, uint32_t* hist, uint32_t* scratch)
+__device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, uint32_t* hist, uint32_t* scratch,
+                                                 int stop_bits = 0)
 {
     constexpr int kSelThreads = NT;
     constexpr int kSelWarps = NT / 32;
@@ -98,8 +101,9 @@ __device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, 
 #pragma unroll
     for (int w = 1; w < kSelWarps; ++w) { lo = min(lo, scratch[w]); hi = max(hi, scratch[kSelWarps + w]); }
     int top = 32 - __clz(hi - lo);   // bits of (key - lo) still undecided
+    const int stop = stop_bits > 0 ? max(top - stop_bits, 0) : 0;
     uint32_t prefix = 0;             // decided high bits of (T - lo)
-    while (top > 0) {
+    while (top > stop) {
         const int shift = max(top - 8, 0), width = top - shift;
         __syncthreads();
         for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
@@ -136,18 +140,17 @@ __device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, 
         krem -= (int)scratch[2 * kSelWarps + 1];
         top = shift;
     }
-    return lo + prefix;
+    return lo + (prefix << top);
 }
 
 // Shared scalars of one selection CTA.
 template <int NT>
-struct SelScalars {
-    uint32_t hist[256];
+struct alignas(16) SelScalars {
+    uint32_t hist[256];   // radix histogram; the emit step reuses it for per-warp 64-bit sums
     uint32_t scratch[2 * (NT / 32) + 2];
     uint32_t count;   // candidates seen by the append pass
     uint32_t base;    // split rows: this CTA's first slot in the row's global buffer
     uint32_t last;    // split rows: this CTA finishes the row
-    uint32_t wgt[NT / 32], weq[NT / 32];
 };
 
 // 1. tau for a row of n > k columns: 0 (every column is a candidate) when n <= buf_cap, else
@@ -173,7 +176,8 @@ __device__ __forceinline__ uint32_t sel_threshold(const float* src, int n, int k
     int rank = (int)ceilf(expect + 4.f * sqrtf(expect) + 4.f);
     rank = min(rank, m);
     __syncthreads();
-    return radix_select<NT>([&](int i) { return sample[i]; }, m, rank, sh.hist, sh.scratch);
+    // 16 bits of the sample's key range are enough: the bin's lower edge only lowers tau a little
+    return radix_select<NT>([&](int i) { return sample[i]; }, m, rank, sh.hist, sh.scratch, 16);
 }
 
 // 2. Appends (key << 32 | column) of every column c in [c0, c1) whose key is >= tau to buf, one
@@ -271,62 +275,51 @@ __device__ __forceinline__ void sel_mark_all(int n, uint32_t* gtmap)
 }
 
 // 4. Emits the marked columns in column order (all of gtmap, the first krem of eqmap), then pads
-// the row to k with -1 (and NaN scores).  Warp w owns bitmap words [w*wpw, (w+1)*wpw).
+// the row to k with -1 (and NaN scores).  Thread t owns a contiguous run of bitmap words; one
+// block-wide scan of its (> T, == T) counts gives both its output offset and its tie rank.
 template <int NT>
 __device__ __forceinline__ void sel_emit(const SelectArgs& a, const RowDesc& rd, int r, const float* src, int n,
                                          int krem, const uint32_t* gtmap, const uint32_t* eqmap, SelScalars<NT>& sh)
 {
-    constexpr int kWarps = NT / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int k = a.k;
     const int nwords = (n + 31) >> 5;
     int32_t* oidx = a.out_idx + (int64_t)r * a.ld_idx;
     float* osc = a.out_score ? a.out_score + (int64_t)r * a.ld_score : nullptr;
-    const int wpw = (nwords + kWarps - 1) / kWarps;
-    const int w0 = warp * wpw, w1 = min(w0 + wpw, nwords);
-    uint32_t gt = 0, eq = 0;
-    for (int w = w0 + lane; w < w1; w += 32) { gt += __popc(gtmap[w]); eq += __popc(eqmap[w]); }
+    const int wpt = (nwords + NT - 1) / NT;
+    const int w0 = min(nwords, tid * wpt), w1 = min(nwords, w0 + wpt);
+    uint32_t ng = 0, ne = 0;
+    for (int w = w0; w < w1; ++w) { ng += __popc(gtmap[w]); ne += __popc(eqmap[w]); }
+    // exclusive scan of (ng, ne) over the threads, packed in 64 bits (each sum < 2^32)
+    const uint64_t mine = ((uint64_t)ng << 32) | ne;
+    uint64_t incl = mine;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        gt += __shfl_xor_sync(0xffffffffu, gt, o);
-        eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
     }
-    if (lane == 0) { sh.wgt[warp] = gt; sh.weq[warp] = eq; }
+    uint64_t* wsum = reinterpret_cast<uint64_t*>(sh.hist);   // NT / 32 <= 32 entries
     __syncthreads();
-    uint32_t eq_rank = 0, out = 0;
-    for (int w = 0; w < warp; ++w) { out += sh.wgt[w]; eq_rank += sh.weq[w]; }
-    out += min(eq_rank, (uint32_t)krem);
-    for (int wb = w0; wb < w1; wb += 32) {
-        const int w = wb + lane;
-        const uint32_t g = w < w1 ? gtmap[w] : 0u, e = w < w1 ? eqmap[w] : 0u;
-        const uint32_t ce = __popc(e);
-        uint32_t pre_e = ce;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t x = __shfl_up_sync(0xffffffffu, pre_e, o);
-            if (lane >= o) pre_e += x;
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    uint64_t before = incl - mine;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    const uint32_t g_before = (uint32_t)(before >> 32), e_before = (uint32_t)before;
+    uint32_t out = g_before + min(e_before, (uint32_t)krem);   // ties before this thread are taken first
+    int left_e = (int)min(ne, (uint32_t)max(0, krem - (int)e_before));
+    for (int w = w0; w < w1; ++w) {
+        uint32_t e = eqmap[w], te = 0;
+        for (; left_e > 0 && e; --left_e) {   // the lowest remaining ties
+            const uint32_t low = e & (0u - e);
+            te |= low;
+            e ^= low;
         }
-        const uint32_t rank0 = eq_rank + pre_e - ce;   // ties before this word
-        const int n_take_e = (int)min(ce, (uint32_t)max(0, krem - (int)rank0));
-        uint32_t take_e = e;
-        for (int drop = (int)ce - n_take_e; drop > 0; --drop) take_e &= ~(1u << (31 - __clz(take_e)));   // keep lowest
-        const uint32_t take = g | take_e;
-        const uint32_t ct = __popc(take);
-        uint32_t pre_t = ct;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t x = __shfl_up_sync(0xffffffffu, pre_t, o);
-            if (lane >= o) pre_t += x;
-        }
-        uint32_t o = out + pre_t - ct;
-        for (uint32_t bits = take; bits; bits &= bits - 1) {
+        for (uint32_t bits = gtmap[w] | te; bits; bits &= bits - 1) {
             const int col = w * 32 + __ffs(bits) - 1;
-            oidx[o] = map_col(a.map, rd, col);
-            if (osc) osc[o] = key_score(score_key(__ldg(src + col)));
-            ++o;
+            oidx[out] = map_col(a.map, rd, col);
+            if (osc) osc[out] = key_score(score_key(__ldg(src + col)));
+            ++out;
         }
-        out += __shfl_sync(0xffffffffu, pre_t, 31);
-        eq_rank += __shfl_sync(0xffffffffu, pre_e, 31);
     }
     const int n_out = min(n, k);
     for (int j = n_out + tid; j < k; j += NT) {
@@ -345,6 +338,8 @@ __global__ void __launch_bounds__(NT) select_stream_kernel(SelectArgs a)
     uint64_t* buf = reinterpret_cast<uint64_t*>(sel_smem + a.sample_bytes);
     uint32_t* gtmap = reinterpret_cast<uint32_t*>(sel_smem + a.sample_bytes + (size_t)cap * 8);
     __shared__ SelScalars<NT> sh;
+    grid_dep_wait();     // the scores come from the previous kernel
+    grid_dep_launch();
 
     const int r = blockIdx.x;
     const RowDesc rd = a.rows[r];
@@ -385,6 +380,8 @@ __global__ void __launch_bounds__(NT) select_split_kernel(SelectArgs a, uint64_t
     uint64_t* buf = reinterpret_cast<uint64_t*>(sel_smem + a.sample_bytes);
     uint32_t* gtmap = reinterpret_cast<uint32_t*>(sel_smem + a.sample_bytes + (size_t)cap * 8);
     __shared__ SelScalars<NT> sh;
+    grid_dep_wait();     // the scores come from the previous kernel
+    grid_dep_launch();
 
     const int r = blockIdx.x / P, p = blockIdx.x % P;
     const RowDesc rd = a.rows[r];

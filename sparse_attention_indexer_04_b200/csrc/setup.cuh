@@ -12,6 +12,7 @@ namespace dsa {
 __global__ void dense_rows_kernel(const int32_t* q_off, const int32_t* k_off, const int32_t* q_pos,
                                   int32_t n_seqs, int32_t n_q, RowDesc* rows)
 {
+    grid_dep_launch();   // the unit builder may launch; it waits for these rows
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= n_q) return;
     const int b = find_seq(q_off, n_seqs, t);
@@ -217,10 +218,6 @@ __global__ void hisa_kept_kernel(const RowDesc* block_rows, const int32_t* mid, 
 }
 
 // ------------------------------------------------------ tensor-core units
-struct TcUnitOut {
-    int32_t row0, nrows, kt0, kt1;
-};
-
 // Work units of one tensor-core scoring launch over launch rows
 // [0, n_rows) = absolute rows [row_base, row_base + n_rows).  Rows are cut into
 // tiles of at most TQ consecutive rows of one segment (seg_off: absolute row
@@ -228,9 +225,12 @@ struct TcUnitOut {
 // Within a segment tiles are emitted last-first, so the longest causal tiles
 // start first.  One CTA of 1024 threads; tile_base is [n_seg + 1] scratch.
 __global__ void tc_units_kernel(const RowDesc* rows, int32_t n_rows, int32_t row_base, const int32_t* seg_off,
-                                int32_t n_seg, int32_t TQ, int32_t splits, int32_t* tile_base, TcUnitOut* units)
+                                int32_t n_seg, int32_t TQ, int32_t splits, const int32_t* k_base, int32_t* tile_base,
+                                TcUnit* units)
 {
     __shared__ int32_t part[1024];
+    grid_dep_wait();     // rows come from the previous kernel
+    grid_dep_launch();   // the scoring kernel may set up while this runs
     const int tid = threadIdx.x, nt = blockDim.x;
     const int per = (n_seg + nt - 1) / nt;   // contiguous segments per thread
     const int s0 = min(n_seg, tid * per), s1 = min(n_seg, s0 + per);
@@ -266,8 +266,10 @@ __global__ void tc_units_kernel(const RowDesc* rows, int32_t n_rows, int32_t row
         int maxnc = 0;
         for (int r = r0; r < r0 + nr; ++r) maxnc = max(maxnc, rows[r].ncols);
         const int nkt = (maxnc + 127) / 128;
+        const RowDesc f = rows[r0];
+        const int krow0 = k_base[f.seq];
         for (int s = 0; s < splits; ++s)
-            units[tau * splits + s] = TcUnitOut{r0, nr, nkt * s / splits, nkt * (s + 1) / splits};
+            units[tau * splits + s] = TcUnit{r0, nr, nkt * s / splits, nkt * (s + 1) / splits, f.qrow, krow0, {0, 0}};
     }
 }
 
