@@ -14,6 +14,7 @@
 #include "score_simt.cuh"
 #include "score_tc.cuh"
 #include "select.cuh"
+#include "reuse.cuh"
 #include "setup.cuh"
 
 using namespace dsa;
@@ -245,21 +246,26 @@ dsa_status set_smem(Kern kern, size_t smem)
                : DSA_ERR_CUDA;
 }
 
+// n_rows_dev (optional): only rows below the count a kernel wrote there are ranked, and each
+// writes output row rows[r].qrow (the one-CTA-per-row kernel only).
 dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, int32_t k, const ColMap& map,
                          const float* S, int64_t ld_s, bool src_from_list, int32_t* out_idx, int64_t ld_idx,
-                         float* out_score, int64_t ld_score, cudaStream_t st, const SelectSplit& sp = SelectSplit{})
+                         float* out_score, int64_t ld_score, cudaStream_t st, const SelectSplit& sp = SelectSplit{},
+                         const int32_t* n_rows_dev = nullptr)
 {
     if (n_rows <= 0) return DSA_OK;
     SelectArgs a{};
     a.rows = rows; a.n_rows = n_rows; a.k = k; a.map = map; a.S = S; a.ld_s = ld_s;
     a.src_from_list = src_from_list ? 1 : 0;
     a.out_idx = out_idx; a.ld_idx = ld_idx; a.out_score = out_score; a.ld_score = ld_score;
+    a.n_rows_dev = n_rows_dev;
+    a.out_from_qrow = n_rows_dev ? 1 : 0;
     a.buf_cap = select_cap(k, max_cols);
     a.sample_bytes = (int32_t)select_sample_bytes(std::max(max_cols, 1));
     const size_t smem = select_smem_bytes(std::max(max_cols, 1), a.buf_cap);
     dsa_status s;
     const int P = select_parts(n_rows, max_cols);
-    if (sp.buf && sp.ctr && n_rows <= sp.max_rows && P > 1) {
+    if (sp.buf && sp.ctr && n_rows <= sp.max_rows && P > 1 && !n_rows_dev) {
         if ((s = set_smem(select_split_kernel<512>, smem)) != DSA_OK) return s;
         DSA_LAUNCH(kProfSelect, st, launch_pdl(true, select_split_kernel<512>, n_rows * P, 512, smem, st, a, sp.buf,
                                                sp.ctr, P));
@@ -456,6 +462,9 @@ dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const
     a.rows = rows;
     a.map = map;
     a.gather = gather ? 1 : 0;
+    // keys are read by several units: gathered candidate lists (shared by a segment's tiles and
+    // by neighbouring segments) and the causal prefixes of prefill (one per query tile)
+    a.keep_keys = gather || tiles > src.n_seqs ? 1 : 0;
     a.W = src.W;
     a.S = S;
     a.ld_s = ld;
@@ -539,7 +548,16 @@ struct PivotPlan {
     TcUnit* units;
     int32_t* tile_base;
     int32_t* group_rows;   // [n_groups + 1] first query row of each group
+    // Reuse: the group's top k + G - 1 candidates, and the queries that need their own selection
+    RowDesc* cand_rows;    // [n_groups]
+    int32_t* gsel;         // [n_groups, kp]
+    float* gscore;         // [n_groups, kp]
+    RowDesc* fb_rows;      // [n_q]
 };
+
+// Reuse's group list length: k plus the most candidates a query of a group with consecutive
+// positions can lose to its own causal limit.
+int32_t reuse_list_len(int32_t k, int32_t G, int32_t C) { return std::min(k + G - 1, C); }
 
 int32_t count_groups(const dsa_batch* b, int32_t G)
 {
@@ -568,7 +586,8 @@ std::vector<int32_t> group_rows_host(const dsa_batch* b, int32_t G)
     return off;
 }
 
-size_t pivot_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t G, int32_t C, PivotPlan* p)
+size_t pivot_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, int32_t G, int32_t C, int32_t mode,
+                  PivotPlan* p)
 {
     Carver c{base};
     const int32_t ng = std::max(1, count_groups(b, G));
@@ -584,7 +603,7 @@ size_t pivot_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t G,
     const int32_t chunk_scan = chunk_rows(ng, ld_scan);
     const size_t s_scan = size_t(chunk_scan) * ld_scan;
     const size_t s_ref = size_t(chunk_rows(std::max(1, b->num_queries), ld_ref)) * ld_ref;
-    p->S = c.take<float>(std::max(s_scan, s_ref));
+    p->S = c.take<float>(mode == 0 ? s_scan : std::max(s_scan, s_ref));
     const std::vector<int32_t> goff = group_offsets_host(b, G);
     const TcSource src{nullptr, 0, nullptr, nullptr, goff.data(), b->num_seqs};
     const std::vector<int32_t> groff = group_rows_host(b, G);
@@ -595,8 +614,23 @@ size_t pivot_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t G,
     p->units = c.take<TcUnit>(cap);
     p->tile_base = c.take<int32_t>(std::max(b->num_seqs, ng) + 1);
     p->group_rows = c.take<int32_t>(ng + 1);
+    p->cand_rows = nullptr;
+    p->gsel = nullptr;
+    p->gscore = nullptr;
+    p->fb_rows = nullptr;
+    if (mode == 0) {
+        const int32_t kp = reuse_list_len(k, G, C);
+        p->cand_rows = c.take<RowDesc>(ng);
+        p->gsel = c.take<int32_t>(size_t(ng) * kp);
+        p->gscore = c.take<float>(size_t(ng) * kp);
+        p->fb_rows = c.take<RowDesc>(std::max(1, b->num_queries));
+    }
     return c.off;
 }
+
+// Count of the Reuse queries left to the per-query selection: a word of the workspace's
+// status area, which every call clears before its first launch.
+int32_t* reuse_fallback_count(void* ws) { return reinterpret_cast<int32_t*>(static_cast<char*>(ws) + 64); }
 
 struct HisaPlan {
     int32_t* block_base;
@@ -756,7 +790,7 @@ size_t pivot_group_index_workspace(const dsa_batch* b, int32_t k, int32_t G, int
     HostInfo hi;
     if (check_batch(b, &hi) != DSA_OK || !pivot_args_ok(k, G, C, mode)) return 0;
     PivotPlan p;
-    return pivot_plan(nullptr, b, hi, G, C, &p);
+    return pivot_plan(nullptr, b, hi, k, G, C, mode, &p);
 }
 
 dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, const float* W, int32_t k,
@@ -770,8 +804,8 @@ dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, c
     if ((s = check_tensors(b, Q, K, W)) != DSA_OK) return s;
     if (b->num_queries > 0 && !idx) return DSA_ERR_INVALID_ARG;
     PivotPlan p;
-    if ((s = check_ws(ws, ws_bytes, pivot_plan(nullptr, b, hi, G, C, &p))) != DSA_OK) return s;
-    pivot_plan(static_cast<char*>(ws), b, hi, G, C, &p);
+    if ((s = check_ws(ws, ws_bytes, pivot_plan(nullptr, b, hi, k, G, C, mode, &p))) != DSA_OK) return s;
+    pivot_plan(static_cast<char*>(ws), b, hi, k, G, C, mode, &p);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((s = clear_status(ws, st)) != DSA_OK) return s;
     const int32_t ng = count_groups(b, G);
@@ -798,8 +832,24 @@ dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, c
     m.list = cand;
     m.list_ld = C;
     if (mode == 0) {
-        // Reuse: rank the group's candidates by their proxy scores inside each query's prefix.
-        return launch_select(p.query_rows, b->num_queries, C, k, m, p.cand_score, C, true, idx, k, nullptr, 0, st);
+        // Reuse: rank the group's candidates by their proxy scores inside each query's prefix.  One
+        // selection of the group's top k + G - 1 serves every query whose prefix keeps k of them;
+        // the others (ragged positions) are ranked one by one.
+        const int32_t kp = reuse_list_len(k, G, C);
+        DSA_LAUNCH(kProfSetup, st, pivot_cand_rows_kernel<<<(ng + 255) / 256, 256, 0, st>>>(p.groups, ng, C, p.cand_rows));
+        if ((s = launched()) != DSA_OK) return s;
+        s = launch_select(p.cand_rows, ng, C, kp, identity_map(), p.cand_score, C, false, p.gsel, kp, p.gscore, kp, st);
+        if (s != DSA_OK) return s;
+        ReuseArgs ra{};
+        ra.groups = p.groups; ra.query_rows = p.query_rows; ra.cand_rows = p.cand_rows;
+        ra.gsel = p.gsel; ra.gscore = p.gscore; ra.kp = kp; ra.k = k; ra.cand = cand; ra.C = C;
+        ra.idx = idx; ra.ld_idx = k; ra.fb_rows = p.fb_rows; ra.fb_count = reuse_fallback_count(ws);
+        const size_t smem = reuse_smem_bytes(kp);
+        if ((s = set_smem(pivot_reuse_kernel, smem)) != DSA_OK) return s;
+        DSA_LAUNCH(kProfSelect, st, pivot_reuse_kernel<<<ng, kReuseThreads, smem, st>>>(ra));
+        if ((s = launched()) != DSA_OK) return s;
+        return launch_select(p.fb_rows, b->num_queries, C, k, m, p.cand_score, C, true, idx, k, nullptr, 0, st,
+                             SelectSplit{}, reuse_fallback_count(ws));
     }
     // Refine: each query scores its eligible candidates with its own indexer (tensor cores,
     // the group's candidate keys gathered tile by tile).

@@ -41,7 +41,7 @@ struct TcArgs {
     ColMap map;              // column -> key index; identity: contiguous key tiles (TMA tile loads),
                              // otherwise each tile's 128 keys are gathered (TMA gather4)
     int32_t gather;          // 0: contiguous tiles, 1: gathered rows
-    int32_t pad2_;
+    int32_t keep_keys;       // 1: other units read the same keys again: load them L2 evict-last
     const float* W;          // row rd.qrow: [H]
     float* S;                // score of launch row r, key s at S[r * ld_s + s]
     int64_t ld_s;
@@ -178,6 +178,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ncmax = __reduce_max_sync(0xffffffffu, ncmax);
         }
         const RowDesc first{0, 0, 0, list};   // map_col reads only the list row
+        const int32_t* lrow = a.gather && a.map.kind != kMapIdentity ? a.map.list + (int64_t)list * a.map.list_ld : nullptr;
+        const bool list4 = a.map.kind == kMapList && (reinterpret_cast<uintptr_t>(lrow) & 15) == 0;
+        const bool block4 = a.map.kind == kMapBlocks && (a.map.block & 3) == 0;
+        // Key rows of this lane's four rows (columns c0 .. c0+3) of tile i: one 16-byte list load,
+        // or one block entry, when the four columns exist.
+        auto tile_rows = [&](int i, int (&y)[4]) {
+            const int c0 = (u.kt0 + i) * 128 + 4 * lane;
+            if (c0 + 3 < ncmax && list4) {
+                const int4 v = __ldg(reinterpret_cast<const int4*>(lrow + c0));
+                y[0] = krow0 + v.x; y[1] = krow0 + v.y; y[2] = krow0 + v.z; y[3] = krow0 + v.w;
+            } else if (c0 + 3 < ncmax && block4) {
+                const int base = krow0 + __ldg(lrow + c0 / a.map.block) * a.map.block + c0 % a.map.block;
+                y[0] = base; y[1] = base + 1; y[2] = base + 2; y[3] = base + 3;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) y[e] = krow0 + map_col(a.map, first, c0 + e < ncmax ? c0 + e : 0);
+            }
+        };
+        // Keys other units read again stay in L2 while the score rows stream out.
+        const uint64_t keep_keys = l2_policy_evict_last();
+        int ynext[4] = {0, 0, 0, 0};   // the next gathered tile's rows, loaded a tile ahead
+        if (a.gather && nkt > 0) tile_rows(0, ynext);
         int stage = 0;
         uint32_t phase = 0;
         int issued = 0;
@@ -189,18 +211,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!a.gather) {
                 if (lane == 0) {
                     const int krow = krow0 + (u.kt0 + i) * 128;
-                    for (int bx = 0; bx < SH::NBOX; ++bx)
-                        tma_load_2d(sK + stage * SH::KTILE + bx * SH::KBOX, &tmK, bx * SH::BOXC, krow, &full[stage]);
+                    for (int bx = 0; bx < SH::NBOX; ++bx) {
+                        if (a.keep_keys)
+                            tma_load_2d_hint(sK + stage * SH::KTILE + bx * SH::KBOX, &tmK, bx * SH::BOXC, krow,
+                                             &full[stage], keep_keys);
+                        else
+                            tma_load_2d(sK + stage * SH::KTILE + bx * SH::KBOX, &tmK, bx * SH::BOXC, krow, &full[stage]);
+                    }
                 }
             } else {
                 __syncwarp();
-                const int c0 = (u.kt0 + i) * 128 + 4 * lane;   // this lane's four rows of the tile
-                int y[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) y[e] = krow0 + map_col(a.map, first, c0 + e < ncmax ? c0 + e : 0);
+                const int y[4] = {ynext[0], ynext[1], ynext[2], ynext[3]};
                 for (int bx = 0; bx < SH::NBOX; ++bx)
-                    tma_gather4_2d(sK + stage * SH::KTILE + bx * SH::KBOX + 4 * lane * SH::ROWB, &tmKg, bx * SH::BOXC,
-                                   y[0], y[1], y[2], y[3], &full[stage]);
+                    tma_gather4_2d_hint(sK + stage * SH::KTILE + bx * SH::KBOX + 4 * lane * SH::ROWB, &tmKg,
+                                        bx * SH::BOXC, y[0], y[1], y[2], y[3], &full[stage], keep_keys);
+                if (i + 1 < nkt) tile_rows(i + 1, ynext);   // in flight while the next slot frees up
             }
             ++issued;
             if (++stage == n_stages) { stage = 0; phase ^= 1u; }
@@ -310,8 +335,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                         for (int h = 0; h < H; ++h) s0 = fmaf(w[h], fmaxf(v[q * H + h], 0.f), s0);
                     }
-                    if (j < u.nrows && key < sNc[j])
-                        a.S[(int64_t)(u.row0 + j) * a.ld_s + key] = (s0 + s1) + 0.f;   // -0 -> +0
+                    if (j < u.nrows && key < sNc[j])   // streaming store: score rows are read once, later
+                        __stcs(&a.S[(int64_t)(u.row0 + j) * a.ld_s + key], (s0 + s1) + 0.f);   // -0 -> +0
                 }
             }
             if (*abort_flag) break;

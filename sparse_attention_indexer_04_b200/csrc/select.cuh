@@ -58,6 +58,9 @@ struct SelectArgs {
     int64_t ld_idx;
     float* out_score;        // nullable, [n_rows, ld_score]
     int64_t ld_score;
+    const int32_t* n_rows_dev;   // nullable: rows [*n_rows_dev, n_rows) are skipped (a count a kernel wrote)
+    int32_t out_from_qrow;       // 1: row r writes output row rows[r].qrow instead of r
+    int32_t pad_;
 };
 
 
@@ -342,6 +345,7 @@ __global__ void __launch_bounds__(NT) select_stream_kernel(SelectArgs a)
     grid_dep_launch();
 
     const int r = blockIdx.x;
+    if (a.n_rows_dev && r >= *a.n_rows_dev) return;   // uniform exit
     const RowDesc rd = a.rows[r];
     const int n = rd.ncols;
     const int k = a.k;
@@ -363,7 +367,7 @@ __global__ void __launch_bounds__(NT) select_stream_kernel(SelectArgs a)
         sel_mark_all<NT>(n, gtmap);
     }
     __syncthreads();
-    sel_emit<NT>(a, rd, r, src, n, krem, gtmap, eqmap, sh);
+    sel_emit<NT>(a, rd, a.out_from_qrow ? rd.qrow : r, src, n, krem, gtmap, eqmap, sh);
 }
 
 // Few long rows: P CTAs per row (blockIdx.x = r * P + p).  Every CTA of a row derives the same

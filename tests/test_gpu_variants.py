@@ -56,6 +56,29 @@ def test_pivot_ragged_integer_exact(mode):
     check_exact_sets(idx, (ref["reuse_idx"] if mode == 0 else ref["refine_idx"])[r], "idx")
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+def test_pivot_random_positions_exact(mode):
+    """Queries of a group at scattered positions: Reuse serves some from the group's shared list and
+    ranks the rest one by one; both must equal the oracle exactly."""
+    b = workloads.ragged(41, [40, 24, 9], [300, 150, 64], H=4, d=32, k=24, integer=True, pos_mode="random")
+    G, C, k = 8, 64, 24
+    idx, cand = Dev(b).pivot(k, G, C, mode)
+    ref = oracle.pivot(b, G, C, k)
+    check_exact_sets(cand, ref["cand"], "cand")
+    check_exact_sets(idx, (ref["reuse_idx"] if mode == 0 else ref["refine_idx"])[group_rows(b, G)], "idx")
+
+
+def test_pivot_reuse_long_groups_exact():
+    """Reuse over a long prefill: groups of 16 consecutive queries, each query dropping up to 15 of the
+    group's k + 15 best candidates; integer inputs with many ties, exact against the oracle."""
+    b = workloads.tiny_integer(seed=9, T=2048, H=4, d=32, k=128)
+    G, C, k = 16, 512, 128
+    idx, cand = Dev(b).pivot(k, G, C, 0)
+    ref = oracle.pivot(b, G, C, k)
+    check_exact_sets(cand, ref["cand"], "cand")
+    check_exact_sets(idx, ref["reuse_idx"][group_rows(b, G)], "idx")
+
+
 def check_pivot_bf16(b, G, C, k, mode):
     idx, cand = Dev(b).pivot(k, G, C, mode)
     own = oracle.pivot(b, G, C, k)                      # the oracle's own two stages
