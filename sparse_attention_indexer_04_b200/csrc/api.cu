@@ -410,10 +410,16 @@ dsa_status launch_tc_shape(const CUtensorMap& mq, const CUtensorMap& mk, const C
     args.n_stages = stages;
     // >= 120 KB keeps one CTA per SM, so no two CTAs ever wait on each other for the 512 TMEM columns.
     const int smem = std::max((int)SH::smem_bytes(n_acc, stages), 120 * 1024);
-    if (cudaFuncSetAttribute(score_tc_kernel<D, H>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return DSA_ERR_CUDA;
-    DSA_LAUNCH(kProfScoreTc, st, launch_pdl(latency_bound(n_units), score_tc_kernel<D, H>, n_units, kTcThreads, smem, st,
-                                            mq, mk, mkg, args));
+    dsa_status s;
+    if (a.gather) {
+        if ((s = set_smem(score_tc_kernel<D, H, true>, smem)) != DSA_OK) return s;
+        DSA_LAUNCH(kProfScoreTc, st, launch_pdl(latency_bound(n_units), score_tc_kernel<D, H, true>, n_units,
+                                                kTcThreads, smem, st, mq, mk, mkg, args));
+    } else {
+        if ((s = set_smem(score_tc_kernel<D, H, false>, smem)) != DSA_OK) return s;
+        DSA_LAUNCH(kProfScoreTc, st, launch_pdl(latency_bound(n_units), score_tc_kernel<D, H, false>, n_units,
+                                                kTcThreadsTiles, smem, st, mq, mk, mkg, args));
+    }
     return launched();
 }
 

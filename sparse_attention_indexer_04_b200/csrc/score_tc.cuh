@@ -15,12 +15,15 @@
 // accumulators of 256 TMEM columns each, so every key tile in shared memory
 // feeds two MMAs — and a range of its key tiles.  Column c of the segment is
 // key map(c): contiguous key tiles are loaded with TMA tile loads, gathered
-// ones with TMA gather4 (four rows per instruction, one per producer lane).
+// ones with TMA gather4 (four rows per instruction and lane).  A warp issues
+// its lanes' gather4 one after another, so a gathered tile (32 * d/64 of them)
+// is split over three producer warps, each with its own full barrier.
 // Roles:
 //   warp 0      TMA producer: the query tile once, then a ring of key tiles
 //   warp 1      TMEM allocator and MMA issuer (one thread)
 //   warps 2..9  epilogue: TMEM -> registers, ReLU, weighted head sum, causal
 //               mask, fp32 score store
+//   warps 10-11 more producers of gathered tiles (idle for contiguous ones)
 // The two accumulators are handed back and forth between MMA and epilogue
 // with mbarriers, so the MMAs into one overlap the epilogue of the other.
 // Every wait is bounded (1 s); a wait that runs out records an error in the
@@ -31,7 +34,9 @@
 
 namespace dsa {
 
-constexpr int kTcThreads = 320;
+constexpr int kTcProducers = 3;   // warps issuing gathered tiles: 0, 10, 11
+constexpr int kTcThreads = 384;   // launches of contiguous tiles use the first 320 (warps 0..9)
+constexpr int kTcThreadsTiles = 320;
 constexpr int kTcMaxStages = 8;
 constexpr uint32_t kErrSmemAlign = 3;
 
@@ -63,7 +68,7 @@ struct TcShape {
     static constexpr uint32_t KTILE = 128u * D * 2;
     static constexpr uint32_t W_BYTES = 2u * NQA * H * 4;
     static constexpr uint32_t NC_BYTES = 2u * NQA * 4;
-    static constexpr uint32_t BAR_BYTES = 256;
+    static constexpr uint32_t BAR_BYTES = 512;
 
     // Q tiles, key stages, W, eligible counts; the barriers and TMEM slot sit in the last
     // BAR_BYTES of the allocation, a place the prologue knows before the unit is read.
@@ -98,12 +103,15 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, uint32_t
     }
 }
 
-template <int D, int H>
-__global__ void __launch_bounds__(kTcThreads, 1)
+// GATHER: the unit's key tiles are gathered through the column map (a.gather == 1).  The two
+// cases are compiled apart, so contiguous tiles keep the single-producer code.
+template <int D, int H, bool GATHER>
+__global__ void __launch_bounds__(GATHER ? kTcThreads : kTcThreadsTiles, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmKg, TcArgs a)
 {
     using SH = TcShape<D, H>;
+    constexpr int NP = GATHER ? kTcProducers : 1;   // producers with a full barrier per stage
     constexpr int NQA = SH::NQA;
     constexpr int QH = NQA / 2;   // queries of one accumulator handled by one epilogue half
 
@@ -113,8 +121,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         return;
     }
     const int n_stages = a.n_stages;
+    // full[p * n_stages + s]: producer p's part of stage s has landed
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + dynamic_smem_size() - SH::BAR_BYTES);
-    uint64_t* empty = full + n_stages;
+    uint64_t* empty = full + NP * n_stages;
     uint64_t* qfull = empty + n_stages;
     uint64_t* tfull = qfull + 1;
     uint64_t* tempty = tfull + 2;
@@ -126,7 +135,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < n_stages; ++i) {
-            mbar_init(&full[i], 1);
+            for (int p = 0; p < NP; ++p) mbar_init(&full[p * n_stages + i], 1);
             mbar_init(&empty[i], 1);
         }
         mbar_init(qfull, 1);
@@ -140,7 +149,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmQ);
-        prefetch_tensormap(a.gather ? &tmKg : &tmK);
+        prefetch_tensormap(GATHER ? &tmKg : &tmK);
     }
     if (warp == 1) tmem_alloc(tmem_slot, 512);
     grid_dep_wait();     // the unit table and rows come from earlier kernels
@@ -160,31 +169,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (!active) {
         // nothing to score: fall through to the TMEM release
-    } else if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
+    } else if (warp == 0 || (GATHER && warp >= 10)) {
+        // ------------------------------------------------------ producers
+        const int pw = warp == 0 ? 0 : warp - 9;   // producer index
         const int krow0 = u.krow0;
-        if (lane == 0) {
+        if (pw == 0 && lane == 0) {
             mbar_arrive_expect_tx(qfull, n_acc * SH::QACC);
             for (int acc = 0; acc < n_acc; ++acc)
                 for (int bx = 0; bx < SH::NBOX; ++bx)
                     tma_load_2d(sQ + acc * SH::QACC + bx * SH::QBOX, &tmQ, bx * SH::BOXC, (u.qrow + acc * NQA) * H,
                                 qfull);
         }
-        // Gathered tiles: the columns of the unit that exist (tiles past them read column 0's key).
+        // Gathered tiles: item w = (box w / 32, rows 4 (w % 32) .. +3) of a tile goes to producer
+        // w % kTcProducers, lane w / kTcProducers.
+        constexpr int kItems = 32 * SH::NBOX;
+        const int w = lane * kTcProducers + pw;
+        const bool has_item = w < kItems;
+        const int rg = w % 32, ibox = w / 32;
+        const uint32_t my_bytes = (uint32_t)((kItems - pw + kTcProducers - 1) / kTcProducers) * 4 * SH::ROWB;
+        uint64_t* my_full = full + pw * n_stages;
+        // the columns of the unit that exist (tiles past them read column 0's key)
         int ncmax = 0, list = 0;
-        if (a.gather) {
+        if (GATHER) {
             list = a.rows[u.row0].list;
             for (int j = lane; j < u.nrows; j += 32) ncmax = max(ncmax, a.rows[u.row0 + j].ncols);
             ncmax = __reduce_max_sync(0xffffffffu, ncmax);
         }
         const RowDesc first{0, 0, 0, list};   // map_col reads only the list row
-        const int32_t* lrow = a.gather && a.map.kind != kMapIdentity ? a.map.list + (int64_t)list * a.map.list_ld : nullptr;
+        const int32_t* lrow = GATHER && a.map.kind != kMapIdentity ? a.map.list + (int64_t)list * a.map.list_ld : nullptr;
         const bool list4 = a.map.kind == kMapList && (reinterpret_cast<uintptr_t>(lrow) & 15) == 0;
         const bool block4 = a.map.kind == kMapBlocks && (a.map.block & 3) == 0;
         // Key rows of this lane's four rows (columns c0 .. c0+3) of tile i: one 16-byte list load,
         // or one block entry, when the four columns exist.
         auto tile_rows = [&](int i, int (&y)[4]) {
-            const int c0 = (u.kt0 + i) * 128 + 4 * lane;
+            const int c0 = (u.kt0 + i) * 128 + 4 * rg;
             if (c0 + 3 < ncmax && list4) {
                 const int4 v = __ldg(reinterpret_cast<const int4*>(lrow + c0));
                 y[0] = krow0 + v.x; y[1] = krow0 + v.y; y[2] = krow0 + v.z; y[3] = krow0 + v.w;
@@ -199,7 +217,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // Keys other units read again stay in L2 while the score rows stream out.
         const uint64_t keep_keys = l2_policy_evict_last();
         int ynext[4] = {0, 0, 0, 0};   // the next gathered tile's rows, loaded a tile ahead
-        if (a.gather && nkt > 0) tile_rows(0, ynext);
+        if (GATHER && has_item && nkt > 0) tile_rows(0, ynext);
         int stage = 0;
         uint32_t phase = 0;
         int issued = 0;
@@ -207,35 +225,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int ok = 1;
             if (lane == 0) ok = tc_wait(&empty[stage], phase ^ 1u, a.status, 1, abort_flag) ? 1 : 0;
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            if (lane == 0) mbar_arrive_expect_tx(&full[stage], SH::KTILE);
-            if (!a.gather) {
+            if constexpr (!GATHER) {
                 if (lane == 0) {
+                    mbar_arrive_expect_tx(&my_full[stage], SH::KTILE);
                     const int krow = krow0 + (u.kt0 + i) * 128;
                     for (int bx = 0; bx < SH::NBOX; ++bx) {
                         if (a.keep_keys)
                             tma_load_2d_hint(sK + stage * SH::KTILE + bx * SH::KBOX, &tmK, bx * SH::BOXC, krow,
-                                             &full[stage], keep_keys);
+                                             &my_full[stage], keep_keys);
                         else
-                            tma_load_2d(sK + stage * SH::KTILE + bx * SH::KBOX, &tmK, bx * SH::BOXC, krow, &full[stage]);
+                            tma_load_2d(sK + stage * SH::KTILE + bx * SH::KBOX, &tmK, bx * SH::BOXC, krow,
+                                        &my_full[stage]);
                     }
                 }
             } else {
+                if (lane == 0) mbar_arrive_expect_tx(&my_full[stage], my_bytes);
                 __syncwarp();
-                const int y[4] = {ynext[0], ynext[1], ynext[2], ynext[3]};
-                for (int bx = 0; bx < SH::NBOX; ++bx)
-                    tma_gather4_2d_hint(sK + stage * SH::KTILE + bx * SH::KBOX + 4 * lane * SH::ROWB, &tmKg,
-                                        bx * SH::BOXC, y[0], y[1], y[2], y[3], &full[stage], keep_keys);
-                if (i + 1 < nkt) tile_rows(i + 1, ynext);   // in flight while the next slot frees up
+                if (has_item) {
+                    const int y[4] = {ynext[0], ynext[1], ynext[2], ynext[3]};
+                    tma_gather4_2d_hint(sK + stage * SH::KTILE + ibox * SH::KBOX + 4 * rg * SH::ROWB, &tmKg,
+                                        ibox * SH::BOXC, y[0], y[1], y[2], y[3], &my_full[stage], keep_keys);
+                    if (i + 1 < nkt) tile_rows(i + 1, ynext);   // in flight while the next slot frees up
+                }
             }
             ++issued;
             if (++stage == n_stages) { stage = 0; phase ^= 1u; }
         }
         // Before leaving, every copy this warp started must have landed.
         if (lane == 0 && *abort_flag) {
-            mbar_wait(qfull, 0, a.status, 10);
+            if (pw == 0) mbar_wait(qfull, 0, a.status, 10);
             for (int back = 1; back <= n_stages && back <= issued; ++back) {
                 const int i = issued - back;
-                mbar_wait(&full[i % n_stages], (uint32_t)((i / n_stages) & 1), a.status, 11);
+                mbar_wait(&my_full[i % n_stages], (uint32_t)((i / n_stages) & 1), a.status, 11);
             }
         }
         __syncwarp();
@@ -255,7 +276,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 uint32_t phase = 0;
                 uint32_t tph[2] = {0, 0};
                 for (int i = 0; i < nkt && !*abort_flag; ++i) {
-                    if (!tc_wait(&full[stage], phase, a.status, 3, abort_flag)) break;
+                    bool landed = true;
+                    for (int p = 0; p < NP && landed; ++p)
+                        landed = tc_wait(&full[p * n_stages + stage], phase, a.status, 3, abort_flag);
+                    if (!landed) break;
                     tc_fence_after();
                     for (int qb = 0; qb < n_acc; ++qb) {
                         // one query block: the two accumulators alternate tile by tile
@@ -285,14 +309,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_wait(drain, 0, a.status, 12);
         }
         __syncwarp();
-    } else {
+    } else {   // warps 2..9
         // ---------------------------------------------------------- epilogue
         // the tile's head weights and eligible counts, shared by the 8 epilogue warps
-        for (int i = threadIdx.x - 64; i < 2 * NQA * H; i += kTcThreads - 64) {
+        for (int i = threadIdx.x - 64; i < 2 * NQA * H; i += 256) {
             const int j = i / H;
             sW[i] = j < u.nrows ? a.W[(int64_t)a.rows[u.row0 + j].qrow * H + (i % H)] : 0.f;
         }
-        for (int j = threadIdx.x - 64; j < 2 * NQA; j += kTcThreads - 64)
+        for (int j = threadIdx.x - 64; j < 2 * NQA; j += 256)
             sNc[j] = j < u.nrows ? a.rows[u.row0 + j].ncols : 0;
         asm volatile("bar.sync 1, 256;" ::: "memory");   // named barrier of the epilogue warps only
         const int quarter = warp & 3;           // TMEM lanes this warp may read
