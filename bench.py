@@ -233,10 +233,12 @@ class Hisa:
                             idx=self.idx, ws=self.ws)
 
 
-def secondary(device, flush, steps):
+def secondary(device, flush, steps, only=None, pivot_T=131072):
     out = {}
 
     def run(name, make, extra):
+        if only and only not in name:
+            return
         try:
             t0 = time.time()
             step = make()
@@ -266,12 +268,13 @@ def secondary(device, flush, steps):
     run("dense_decode_B16_L32768_mtp2", lambda: DenseTopk(workloads.dense_decode(seed=1), device), dec_extra)
     run("dense_decode_B16_L131072_mtp2", lambda: DenseTopk(workloads.dense_decode(seed=1, L=131072), device),
         dec_extra)
-    pv = workloads.pivot_prefill(seed=3)
-    dense_pairs = pv.eligible_pairs()
-    for mode, name in ((0, "reuse"), (1, "refine")):
-        run(f"pivot_prefill_T131072_G16_C8192_{name}", lambda m=mode: Pivot(pv, device, m),
-            lambda step, ms: {"dense_equiv_gpairs_s": round(dense_pairs / (ms * 1e-3) / 1e9, 2)})
-    del pv
+    if not only or "pivot" in only or "reuse" in only or "refine" in only:
+        pv = workloads.pivot_prefill(seed=3, T=pivot_T)
+        dense_pairs = pv.eligible_pairs()
+        for mode, name in ((0, "reuse"), (1, "refine")):
+            run(f"pivot_prefill_T{pivot_T}_G16_C8192_{name}", lambda m=mode: Pivot(pv, device, m),
+                lambda step, ms: {"dense_equiv_gpairs_s": round(dense_pairs / (ms * 1e-3) / 1e9, 2)})
+        del pv
     run("hisa_decode_B4_L262144_keep64", lambda: Hisa(workloads.hisa_decode(seed=4), device), lambda s, ms: {})
     return out
 
@@ -336,11 +339,20 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--secondary-steps", type=int, default=5)
     ap.add_argument("--T", type=int, default=32768, help="prefill length (smaller only for profiling captures)")
+    ap.add_argument("--only", default=None,
+                    help="profiling: run only the secondary workloads whose name contains this (no headline line)")
+    ap.add_argument("--pivot-T", type=int, default=131072, help="PIVOT prefill length (smaller for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.only:
+        device = torch.device("cuda", 0)
+        torch.cuda.set_device(device)
+        sec = secondary(device, L2Flush(device), args.secondary_steps, args.only, args.pivot_T)
+        print(json.dumps({"secondary": sec}))
         return
 
     world, rank, local = dist_setup()
@@ -413,6 +425,22 @@ def step_pairs(b):
     return b.eligible_pairs()
 
 
+def measured_traffic(kernel):
+    """DRAM bytes per launch of `kernel` on the 32K prefill from the committed ncu capture, or None when
+    the kernel's sources changed since (the capture no longer describes it)."""
+    import hashlib
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "dram_traffic_dense_prefill_32k.json")
+    try:
+        rec = json.load(open(path))["kernels"][kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "sparse_attention_indexer_04_b200", "csrc")
+    m = hashlib.sha256()
+    for f in rec["sources"]:
+        m.update(open(os.path.join(src, f), "rb").read())
+    return rec["bytes_per_launch"] if m.hexdigest() == rec["sources_sha256"] else None
+
+
 def roofline_entries(prof, step, b, steps, peaks, peaks_src):
     """Per-kernel roofline from the live per-kernel event times; the dominant (most time) is the headline.
 
@@ -447,7 +475,9 @@ def roofline_entries(prof, step, b, steps, peaks, peaks_src):
             out.append(e)
             continue
         e["frac"] = round(e["achieved"] / e["peak"], 4)
-        e["traffic"] = None
+        # DRAM bytes per launch (ncu), beside the algorithmic work per launch
+        e["traffic"] = measured_traffic(name) if b.n_q == 32768 else None
+        e["alg_per_launch"] = round(e["alg_per_step"] / max(1.0, n / steps))
         out.append(e)
     out.sort(key=lambda e: -e["ms_per_step"])
     dom = next(e for e in out if "bound" in e)
