@@ -69,11 +69,23 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest x over all ranks (device times: the job takes as long as its slowest rank)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(rank: int, T: int):
+    """Rank r's own prefill sequence (weak scaling: independent sequences, no data exchange)."""
+    return workloads.dense_prefill(seed=2 + 1000 * rank, T=T)
+
+
+def job_value(pairs_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job Gpairs/s: every rank's pairs over the slowest rank's step time."""
+    return pairs_per_rank * world / (ms_per_step * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------- clocks
@@ -361,7 +373,7 @@ def main():
     import sparse_attention_indexer_04_b200 as dsa
 
     peaks, peaks_src = load_peaks()
-    b = workloads.dense_prefill(seed=2 + 1000 * rank, T=args.T)
+    b = rank_workload(rank, args.T)
     step = DenseTopk(b, device)
     flush = L2Flush(device)
     for _ in range(args.warmup):
@@ -379,7 +391,7 @@ def main():
     torch.cuda.synchronize()
     total_ms = max_over_ranks(sum(ms), world)
     ms_per_step = total_ms / args.steps
-    value = step.pairs * world / (ms_per_step * 1e-3) / 1e9
+    value = job_value(step.pairs, world, ms_per_step)
 
     # ---- per-kernel times over a second pass of the same steps (events on the launching stream)
     dsa.profile_enable(True)
@@ -389,7 +401,7 @@ def main():
     roof, kernels = roofline_entries(prof, step, b, args.steps, peaks, peaks_src)
 
     e2e_ms, h2d, d2h = step.e2e(max(2, args.steps // 2), flush)
-    e2e = {"value": step.pairs * world / (max_over_ranks(e2e_ms, world) * 1e-3) / 1e9, "unit": "Gpairs/s",
+    e2e = {"value": job_value(step.pairs, world, max_over_ranks(e2e_ms, world)), "unit": "Gpairs/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None

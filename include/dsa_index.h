@@ -180,6 +180,21 @@ dsa_status hisa_index(const dsa_batch* batch, const void* Q, const void* K, cons
 dsa_status dsa_device_check(void* ws, void* stream, uint32_t* detail);
 
 /* --------------------------------------------------------------------
+ * Self-test of the bounded waits (no counterpart in the pages; a check of
+ * this library's failure reporting).  Every wait of the library's kernels on
+ * an mbarrier gives up after a time limit (1 s), records code 1 (wait ran
+ * out) in the workspace status word and lets the kernel finish.  This call
+ * launches one CTA that waits, through the same wait routine, on a barrier
+ * nothing ever completes, with a limit of `limit_us` microseconds
+ * (1 .. 1000000): the wait runs out, the kernel records code 1 and returns,
+ * and the context stays usable.  A later dsa_device_check on the same stream
+ * reports DSA_ERR_DEVICE_CHECK with detail 1.  `ws` needs 256 bytes; the
+ * call clears its status word first.  DSA_ERR_INVALID_ARG for a null or
+ * misaligned `ws`, a short `ws_bytes` or a limit outside the range.
+ */
+dsa_status dsa_selftest_wait_timeout(uint32_t limit_us, void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------
  * Allocation-free dense top-k (no counterpart in the pages; a convenience of
  * this library).  Same computation, arguments and outputs as dsa_index_topk,
  * but the workspace is a device array inside the library, for callers that

@@ -70,6 +70,7 @@ _sig("hisa_pool_keys", ctypes.c_int, _B, _P, _I32, _P, _P)
 _sig("hisa_index_workspace", _SZ, _B, _I32, _I32, _I32)
 _sig("hisa_index", ctypes.c_int, _B, _P, _P, _P, _P, _I32, _I32, _I32, _P, _P, _P, _SZ, _P)
 _sig("dsa_device_check", ctypes.c_int, _P, _P, ctypes.POINTER(ctypes.c_uint32))
+_sig("dsa_selftest_wait_timeout", ctypes.c_int, ctypes.c_uint32, _P, _SZ, _P)
 _sig("dsa_index_topk_static_capacity", _SZ)
 _sig("dsa_index_topk_static", ctypes.c_int, _B, _P, _P, _P, _I32, _P, _P, _P)
 _sig("dsa_profile_enable", None, _I32)
@@ -267,6 +268,13 @@ def profile_read():
     if kinds < 0:
         raise DsaError(4, "dsa_profile_read")
     return {_lib.dsa_profile_kind_name(i).decode(): (float(ms[i]), int(n[i])) for i in range(kinds) if n[i]}
+
+
+def selftest_wait_timeout(limit_us: int, ws, stream=None):
+    """Launch the bounded-wait self-test: a wait nothing completes runs out after limit_us and records
+    code 1 in ws's status word (read it with device_check)."""
+    _check(_lib.dsa_selftest_wait_timeout(limit_us, _ptr(ws), _bytes(ws), _stream(stream)),
+           "dsa_selftest_wait_timeout")
 
 
 def device_check(ws, stream=None) -> int:

@@ -931,9 +931,8 @@ dsa_status hisa_index(const dsa_batch* b, const void* Q, const void* K, const fl
     int32_t* kept = kept_out ? kept_out : p.kept;
     const unsigned g = (nq + 255) / 256;
 
-    DSA_LAUNCH(kProfSetup, st, hisa_block_base_kernel<<<1, 32, 0, st>>>(b->k_offsets, b->num_seqs, B, p.block_base));
-    DSA_LAUNCH(kProfSetup, st, hisa_block_rows_kernel<<<g, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos, b->num_seqs, nq, B,
-                                              p.block_rows));
+    DSA_LAUNCH(kProfSetup, st, hisa_setup_kernel<<<(nq + 256) / 256, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos,
+                                                    b->num_seqs, nq, B, p.block_base, p.block_rows, p.query_off));
     if ((s = launched()) != DSA_OK) return s;
     // Coarse stage: middle blocks scored on their pooled keys, top `keep` kept.
     const int32_t max_mid = std::max(0, (hi.max_k + B - 1) / B - 2);
@@ -949,8 +948,6 @@ dsa_status hisa_index(const dsa_batch* b, const void* Q, const void* K, const fl
     m.block = B;
     m.list = kept;
     m.list_ld = keep + 2;
-    DSA_LAUNCH(kProfSetup, st, iota_kernel<<<(nq + 256) / 256, 256, 0, st>>>(p.query_off, nq));
-    if ((s = launched()) != DSA_OK) return s;
     const std::vector<int32_t> qoff = iota_host(nq);
     const TcSource src{Q, nq, W, p.query_off, qoff.data(), nq};
     return tc_score_and_select(p.token_rows, nq, src, H, D, K, b->num_keys, b->k_offsets, m, (keep + 2) * B, p.S,
@@ -1000,6 +997,17 @@ int32_t dsa_profile_read(float* ms, int32_t* launches, int32_t cap)
 }
 
 // ------------------------------------------------------------ device check
+dsa_status dsa_selftest_wait_timeout(uint32_t limit_us, void* ws, size_t ws_bytes, void* stream)
+{
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255) || ws_bytes < kStatusBytes) return DSA_ERR_INVALID_ARG;
+    if (limit_us < 1 || limit_us > 1000000) return DSA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, kStatusBytes, st) != cudaSuccess) return DSA_ERR_CUDA;
+    DSA_LAUNCH(kProfSetup, st, selftest_wait_kernel<<<1, 32, 0, st>>>(static_cast<uint32_t*>(ws),
+                                                                      uint64_t(limit_us) * 1000u));
+    return launched();
+}
+
 dsa_status dsa_device_check(void* ws, void* stream, uint32_t* detail)
 {
     if (!ws) return DSA_ERR_INVALID_ARG;

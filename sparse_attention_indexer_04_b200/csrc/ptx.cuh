@@ -66,7 +66,8 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity)
 // workspace status word and returns false.  Never spins forever.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s; every wait here is for work of the same CTA
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status, uint32_t where)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status, uint32_t where,
+                                          uint64_t limit_ns = kWaitLimitNs)
 {
     if (mbar_test(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
@@ -74,11 +75,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
 #pragma unroll 1
         for (int i = 0; i < 256; ++i)
             if (mbar_test(bar, parity)) return true;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             record_error(status, kErrWaitTimeout, where);
             return false;
         }
     }
+}
+
+// One CTA waits, through mbar_wait, on a barrier nothing completes: the wait
+// runs out after limit_ns and records kErrWaitTimeout (the library's
+// failure-reporting self-test).
+__global__ void selftest_wait_kernel(uint32_t* status, uint64_t limit_ns)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    mbar_wait(&bar, 0, status, 0, limit_ns);   // no arrival ever comes
 }
 
 // ------------------------------------------------------------------- TMA

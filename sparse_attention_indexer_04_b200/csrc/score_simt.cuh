@@ -3,8 +3,9 @@
 // Used where the operand is not a bf16 tensor-core tile: HISA's pooled fp32
 // block keys, and small or irregular rows.  One CTA scores one row against
 // 128 consecutive columns; thread c holds its key in registers and walks
-// the row's H heads, I = sum_h w_h * max(0, q_h . k), the dot products
-// accumulated in fp32 in index order.
+// the row's H heads, I = sum_h w_h * max(0, q_h . k), each dot product
+// accumulated in fp32 as four interleaved partial sums (four independent
+// FMA chains instead of one 128-long chain).
 #pragma once
 
 #include "common.cuh"
@@ -78,18 +79,19 @@ __global__ void __launch_bounds__(kSimtCols) score_simt_kernel(ScoreArgs a)
         float kr[D];
         load_key<D>(kp, kr);
         float acc = 0.f;
+#pragma unroll 2
         for (int h = 0; h < a.H; ++h) {
             const float4* qh = reinterpret_cast<const float4*>(sq + h * D);
-            float dot = 0.f;
+            float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
 #pragma unroll
             for (int i = 0; i < D / 4; ++i) {
                 const float4 qv = qh[i];
-                dot = fmaf(qv.x, kr[4 * i], dot);
-                dot = fmaf(qv.y, kr[4 * i + 1], dot);
-                dot = fmaf(qv.z, kr[4 * i + 2], dot);
-                dot = fmaf(qv.w, kr[4 * i + 3], dot);
+                d0 = fmaf(qv.x, kr[4 * i], d0);
+                d1 = fmaf(qv.y, kr[4 * i + 1], d1);
+                d2 = fmaf(qv.z, kr[4 * i + 2], d2);
+                d3 = fmaf(qv.w, kr[4 * i + 3], d3);
             }
-            acc = fmaf(sw[h], fmaxf(dot, 0.f), acc);
+            acc = fmaf(sw[h], fmaxf((d0 + d1) + (d2 + d3), 0.f), acc);
         }
         out = acc + 0.f;   // -0 -> +0
     }

@@ -132,19 +132,6 @@ __global__ void pivot_query_rows_kernel(const int32_t* q_off, const int32_t* k_o
 // HISA ("HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse
 // Attention", abstract): pooled block keys, block filter, token refinement.
 
-// Single CTA: block_base[b] = pooled blocks before sequence b.
-__global__ void hisa_block_base_kernel(const int32_t* k_off, int32_t n_seqs, int32_t B, int32_t* block_base)
-{
-    if (threadIdx.x == 0 && blockIdx.x == 0) {
-        int32_t acc = 0;
-        for (int b = 0; b < n_seqs; ++b) {
-            block_base[b] = acc;
-            acc += (k_off[b + 1] - k_off[b] + B - 1) / B;
-        }
-        block_base[n_seqs] = acc;
-    }
-}
-
 // Pooled key of block j: mean of its keys (fp32 sum in token order).  One
 // CTA of D threads per block; thread i owns dimension i (coalesced rows).
 // The owning sequence is found by walking the key offsets (few sequences).
@@ -176,13 +163,25 @@ __global__ void hisa_pool_kernel(const __nv_bfloat16* K, const int32_t* k_off, i
     }
 }
 
-// Block-scoring rows: the middle blocks 1 .. last-1 of query t (column c is
-// block c + 1).
-__global__ void hisa_block_rows_kernel(const int32_t* q_off, const int32_t* k_off, const int32_t* q_pos,
-                                       int32_t n_seqs, int32_t n_q, int32_t B, RowDesc* rows)
+// HISA set-up in one launch: every CTA writes the block-scoring rows (the
+// middle blocks 1 .. last-1 of query t; column c is block c + 1) and the
+// per-query segment offsets query_off[t] = t of its queries; CTA 0 also
+// writes block_base (first pooled block of each sequence).
+__global__ void hisa_setup_kernel(const int32_t* q_off, const int32_t* k_off, const int32_t* q_pos, int32_t n_seqs,
+                                  int32_t n_q, int32_t B, int32_t* block_base, RowDesc* rows, int32_t* query_off)
 {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        int32_t acc = 0;
+        for (int b = 0; b < n_seqs; ++b) {
+            block_base[b] = acc;
+            acc += (k_off[b + 1] - k_off[b] + B - 1) / B;
+        }
+        block_base[n_seqs] = acc;
+    }
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= n_q) return;
+    if (t > n_q) return;
+    query_off[t] = t;
+    if (t == n_q) return;
     const int b = find_seq(q_off, n_seqs, t);
     const int n = eligible_count(q_pos[t], k_off[b + 1] - k_off[b]);
     const int last = n > 0 ? (n - 1) / B : 0;
@@ -273,8 +272,8 @@ __global__ void tc_units_kernel(const RowDesc* rows, int32_t n_rows, int32_t row
     }
 }
 
-// Row offsets of PIVOT groups (segment g = rows [off[g], off[g+1])) and of
-// single-query segments (off[t] = t), for the tensor-core unit builder.
+// Row offsets of PIVOT groups (segment g = rows [off[g], off[g+1])), for the
+// tensor-core unit builder.
 __global__ void group_row_offsets_kernel(const GroupDesc* groups, int32_t n_groups, int32_t n_q, int32_t* off)
 {
     const int g = blockIdx.x * blockDim.x + threadIdx.x;
@@ -282,11 +281,6 @@ __global__ void group_row_offsets_kernel(const GroupDesc* groups, int32_t n_grou
     if (g == 0) off[n_groups] = n_q;
 }
 
-__global__ void iota_kernel(int32_t* off, int32_t n)
-{
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i <= n) off[i] = i;
-}
 
 // Fills a row-major [rows, cols] fp32 matrix with -inf (masked scores).
 __global__ void fill_neg_inf_kernel(float* S, int64_t ld, int32_t rows, int32_t cols)

@@ -100,6 +100,15 @@ def test_argument_errors_return_before_any_launch():
     assert call_topk(host_layout([1], [1_000_000]), k=2048) == 2
 
 
+def test_selftest_argument_errors_need_no_gpu():
+    lib = dsa.library()
+    P = ctypes.c_void_p
+    assert lib.dsa_selftest_wait_timeout(1000, None, 256, None) == 1
+    assert lib.dsa_selftest_wait_timeout(1000, P(0x10010), 256, None) == 1     # misaligned
+    assert lib.dsa_selftest_wait_timeout(1000, P(0x10000), 16, None) == 1      # too small
+    assert lib.dsa_selftest_wait_timeout(0, P(0x10000), 256, None) == 1        # limit out of range
+
+
 def test_pivot_and_hisa_argument_errors():
     lay = host_layout([8], [8])
     lib = dsa.library()

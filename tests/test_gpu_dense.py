@@ -105,6 +105,15 @@ def test_full_size_decode_32k():
     check_tolerance_rows(idx, ref["idx"], ref["all"])
 
 
+def test_full_size_decode_128k():
+    """Dense decode, 16 sequences x 128K keys, 2 MTP queries each (the decode metric's size): every row."""
+    b = workloads.dense_decode(seed=1, L=131072)
+    idx = Dev(b).topk(2048)
+    ascending_packed(idx)
+    ref = oracle.dense(b, k=2048, want_all=True)
+    check_tolerance_rows(idx, ref["idx"], ref["all"])
+
+
 def test_full_size_prefill_32k_sampled_rows():
     """Dense prefill T = L = 32K, H=64, d=128, k=2048: the whole batch on the GPU, sampled rows checked."""
     b = workloads.dense_prefill(seed=2)

@@ -79,34 +79,43 @@ def test_pivot_reuse_long_groups_exact():
     check_exact_sets(idx, ref["reuse_idx"][group_rows(b, G)], "idx")
 
 
-def check_pivot_bf16(b, G, C, k, mode):
-    idx, cand = Dev(b).pivot(k, G, C, mode)
-    own = oracle.pivot(b, G, C, k)                      # the oracle's own two stages
-    ext = oracle.pivot(b, G, C, k, ext_cand=cand)       # its second stage on the GPU's candidates
-    ascending_packed(cand)
+def check_pivot_bf16(b, G, C, k, mode, groups=None, gpu=None):
+    """bf16 PIVOT against the oracle: stage 1 (candidates) under the tolerance rule, stage 2 against the
+    oracle's second stage on the GPU's own candidates.  `groups`: check only these groups (global group
+    indices of a single-sequence batch); `gpu`: (idx, cand) already computed."""
+    idx, cand = gpu if gpu is not None else Dev(b).pivot(k, G, C, mode)
+    sel = list(range(cand.shape[0])) if groups is None else list(groups)
+    own = oracle.pivot(b, G, C, k, groups=sel)                      # the oracle's own two stages
+    ext = oracle.pivot(b, G, C, k, groups=sel, ext_cand=cand[sel])  # its second stage on the GPU's candidates
+    gc = cand[sel].copy()
+    ascending_packed(gc)
     # stage 1: candidate sets under the rule, scored by the oracle's proxy
-    for g in range(cand.shape[0]):
+    for i, g in enumerate(sel):
         sc = {}
         for src in (own, ext):
-            v = src["cand"][g] >= 0
-            sc.update(zip(src["cand"][g][v].tolist(), src["cand_score"][g][v].tolist()))
-        rms = float(np.sqrt(np.mean(own["cand_score"][g][own["cand"][g] >= 0] ** 2)))
-        msg = check_tolerance_row(cand[g], own["cand"][g], lambda ix: np.array([sc[x] for x in ix]), rms)
+            v = src["cand"][i] >= 0
+            sc.update(zip(src["cand"][i][v].tolist(), src["cand_score"][i][v].tolist()))
+        rms = float(np.sqrt(np.mean(own["cand_score"][i][own["cand"][i] >= 0] ** 2)))
+        msg = check_tolerance_row(gc[i], own["cand"][i], lambda ix: np.array([sc[x] for x in ix]), rms)
         assert msg is None, f"group {g} candidates: {msg}"
     # stage 2: each query against the oracle's second stage on the same candidates
     rows = group_rows(b, G)
+    pos = {g: i for i, g in enumerate(sel)}
     for t in range(b.n_q):
         g = rows[t] // G
-        v = (ext["cand"][g] >= 0) & (ext["cand"][g] <= int(b.q_pos[t]))
-        elig = ext["cand"][g][v]
+        if g not in pos:
+            continue
+        i, j = pos[g], rows[t] % G
+        v = (ext["cand"][i] >= 0) & (ext["cand"][i] <= int(b.q_pos[t]))
+        elig = ext["cand"][i][v]
         if mode == 0:
-            prox = dict(zip(elig.tolist(), ext["cand_score"][g][v].tolist()))
+            prox = dict(zip(elig.tolist(), ext["cand_score"][i][v].tolist()))
             score_of = lambda ix, d=prox: np.array([d[x] for x in ix])
-            ref_row = ext["reuse_idx"][rows[t]]
+            ref_row = ext["reuse_idx"][i * G + j]
         else:
             own_sc = dict(zip(elig.tolist(), oracle.pair_scores(b, [t] * elig.size, elig).tolist()))
             score_of = lambda ix, d=own_sc: np.array([d[x] for x in ix])
-            ref_row = ext["refine_idx"][rows[t]]
+            ref_row = ext["refine_idx"][i * G + j]
         fin = score_of(elig) if elig.size else np.zeros(1)
         rms = float(np.sqrt(np.mean(fin ** 2)))
         msg = check_tolerance_row(idx[t], ref_row, score_of, rms)
@@ -124,6 +133,20 @@ def test_pivot_decode_groups_are_mtp_steps(mode):
     """Decode: a group is the MTP queries of one step (group size = queries per sequence)."""
     b = workloads.dense_decode(seed=32, B=4, L=2000, n_mtp=2, H=64, d=128, k=128)
     check_pivot_bf16(b, G=2, C=512, k=128, mode=mode)
+
+
+def test_full_size_pivot_128k_sampled_groups():
+    """PIVOT at 128K (G = 16, C = 8192, k = 2048): the whole batch on the GPU in both modes; sampled
+    groups (early ones whose prefix is shorter than C, middle and last) checked against the oracle."""
+    b = workloads.pivot_prefill(seed=3)
+    G, C, k = 16, 8192, 2048
+    groups = [0, 3, 600, 4095, 8190, 8191]
+    dev = Dev(b)
+    reuse = dev.pivot(k, G, C, 0)
+    refine = dev.pivot(k, G, C, 1)
+    assert np.array_equal(reuse[1], refine[1])            # both modes share the candidate stage
+    check_pivot_bf16(b, G, C, k, 0, groups=groups, gpu=reuse)
+    check_pivot_bf16(b, G, C, k, 1, groups=groups, gpu=refine)
 
 
 # ------------------------------------------------------------------- HISA
