@@ -437,9 +437,9 @@ def step_pairs(b):
     return b.eligible_pairs()
 
 
-def measured_traffic(kernel):
+def measured_traffic(kernel, launches_per_step):
     """DRAM bytes per launch of `kernel` on the 32K prefill from the committed ncu capture, or None when
-    the kernel's sources changed since (the capture no longer describes it)."""
+    the kernel's sources or its launches per step changed since (the capture no longer describes it)."""
     import hashlib
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "dram_traffic_dense_prefill_32k.json")
     try:
@@ -450,7 +450,8 @@ def measured_traffic(kernel):
     m = hashlib.sha256()
     for f in rec["sources"]:
         m.update(open(os.path.join(src, f), "rb").read())
-    return rec["bytes_per_launch"] if m.hexdigest() == rec["sources_sha256"] else None
+    same = m.hexdigest() == rec["sources_sha256"] and rec.get("launches_per_step") == launches_per_step
+    return rec["bytes_per_launch"] if same else None
 
 
 def roofline_entries(prof, step, b, steps, peaks, peaks_src):
@@ -488,7 +489,7 @@ def roofline_entries(prof, step, b, steps, peaks, peaks_src):
             continue
         e["frac"] = round(e["achieved"] / e["peak"], 4)
         # DRAM bytes per launch (ncu), beside the algorithmic work per launch
-        e["traffic"] = measured_traffic(name) if b.n_q == 32768 else None
+        e["traffic"] = measured_traffic(name, n / steps) if b.n_q == 32768 else None
         e["alg_per_launch"] = round(e["alg_per_step"] / max(1.0, n / steps))
         out.append(e)
     out.sort(key=lambda e: -e["ms_per_step"])

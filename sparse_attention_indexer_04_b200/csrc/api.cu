@@ -23,7 +23,10 @@ namespace {
 
 constexpr int32_t kMaxK = 16384;
 constexpr int32_t kMaxCand = 16384;
-constexpr size_t kScoreBudget = size_t(256) << 20;   // bytes of materialised score rows per launch
+// Bytes of materialised score rows per launch: 1 GiB keeps a 32K prefill's scoring launches at
+// ~1000 units (about 7 waves of 148 SMs), where 256 MiB (256 units, 1.7 waves) lost ~14 % to
+// the last wave.
+constexpr size_t kScoreBudget = size_t(1024) << 20;   // bytes of materialised score rows per launch
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -198,9 +201,10 @@ dsa_status launch_score(const RowDesc* rows, int32_t n_rows, int32_t max_cols, c
 }
 
 // Threads per row of the streaming select: 256 when rows fill the GPU several times over, 512
-// when there are few rows (each row's phases are latency-bound).  Measured on the 32K prefill
-// (32768 rows: 256 best) and the 16 x 32K decode (32 rows: 512 best).
-int select_threads(int32_t n_rows) { return n_rows < 2 * 148 ? 512 : 256; }
+// when there are few rows or k is large (each row's phases are latency-bound).  Measured on the
+// 32K prefill (32768 rows: 256 best), the 16 x 32K decode (32 rows: 512 best) and PIVOT's top-8192
+// candidate selection (512 best).
+int select_threads(int32_t n_rows, int32_t k) { return n_rows < 2 * 148 || k >= 4096 ? 512 : 256; }
 
 // Candidate buffer entries of the select: 1.75 k, or what fits in shared memory next to the
 // bitmaps of max_cols columns (a smaller buffer only sends more rows down the full-row path).
@@ -271,7 +275,7 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
                                                sp.ctr, P));
         return launched();
     }
-    switch (select_threads(n_rows)) {
+    switch (select_threads(n_rows, k)) {
     case 512:
         if ((s = set_smem(select_stream_kernel<512>, smem)) != DSA_OK) return s;
         DSA_LAUNCH(kProfSelect, st, launch_pdl(latency_bound(n_rows), select_stream_kernel<512>, n_rows, 512, smem, st, a));

@@ -78,9 +78,12 @@ __host__ __device__ inline size_t select_smem_bytes(int max_cols, int buf_cap)
 // holding rank `krem` (1 = largest) and, in krem, how many keys equal to T
 // that rank reaches.  Digits are taken from (key - min), starting at the
 // highest bit where min and max differ, 8 bits at a time, so even the first
-// pass spreads the keys over many bins.  With stop_bits > 0 only the top
-// stop_bits bits of (key - min) are resolved and the lower edge of that bin
-// is returned: a key <= T (krem is then meaningless).  All threads call it.
+// pass spreads the keys over many bins.  When the rank falls in a bin whose
+// keys are all taken, the passes stop there and the result says "every key
+// >= the bin's lower edge": T = that edge - 1 and krem = 0 (no tie at T is
+// taken).  With stop_bits > 0 only the top stop_bits bits of (key - min) are
+// resolved and the lower edge of that bin is returned: a key <= T (krem is
+// then meaningless).  All threads call it.
 template <int NT, typename Get>
 __device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, uint32_t* hist, uint32_t* scratch,
                                                  int stop_bits = 0)
@@ -136,12 +139,20 @@ __device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, 
                 }
                 scratch[2 * kSelWarps] = 8 * lane + b;
                 scratch[2 * kSelWarps + 1] = acc;
+                scratch[2 * kSelWarps + 2] = acc + c[b] == (uint32_t)krem;   // the whole bin is taken
             }
         }
         __syncthreads();
         prefix = (prefix << width) | scratch[2 * kSelWarps];
         krem -= (int)scratch[2 * kSelWarps + 1];
         top = shift;
+        if (stop_bits == 0 && top > 0 && scratch[2 * kSelWarps + 2]) {
+            const uint32_t edge = lo + (prefix << top);   // lowest key the bin can hold
+            if (edge > 0) {
+                krem = 0;
+                return edge - 1;
+            }
+        }
     }
     return lo + (prefix << top);
 }
@@ -150,7 +161,7 @@ __device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, 
 template <int NT>
 struct alignas(16) SelScalars {
     uint32_t hist[256];   // radix histogram; the emit step reuses it for per-warp 64-bit sums
-    uint32_t scratch[2 * (NT / 32) + 2];
+    uint32_t scratch[2 * (NT / 32) + 4];
     uint32_t count;   // candidates seen by the append pass
     uint32_t base;    // split rows: this CTA's first slot in the row's global buffer
     uint32_t last;    // split rows: this CTA finishes the row
