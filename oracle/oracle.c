@@ -349,7 +349,9 @@ static void pivot_group(void* p, int64_t gi)
 
     /* One shared scan over the prefix up to the group's last position. */
     int64_t n_scan = eligible_count(p_last, L);
-    scored_t* cand = (scored_t*)malloc(sizeof(scored_t) * (size_t)(n_scan > 0 ? n_scan : 1));
+    /* room for the scanned keys, or for C supplied candidates (they may lie past p_last) */
+    int64_t n_room = n_scan > C ? n_scan : C;
+    scored_t* cand = (scored_t*)malloc(sizeof(scored_t) * (size_t)(n_room > 0 ? n_room : 1));
     int64_t n_cand;
     if (c->ext_cand) {
         n_cand = 0;
