@@ -150,6 +150,26 @@ dsa_status pivot_group_index(const dsa_batch* batch, const void* Q, const void* 
                              int32_t* cand, void* ws, size_t ws_bytes, void* stream);
 
 /* --------------------------------------------------------------------
+ * Refine on supplied candidates: the second stage of PIVOT Refine over the
+ * caller's candidate lists instead of a proxy scan - a selection made once
+ * and refined by others, as the followers of an anchor layer ("LatentIndex",
+ * abstract) or a group's token bank ("ADIndex: Layer-Adaptive Sparse
+ * Attention Indexing via Group-Level Distillation", abstract).
+ * Groups as in pivot_group_index.  cand [n_groups, n_cand] int32 (device,
+ * read only): group g's candidates, sequence-local key indices, strictly
+ * ascending, then -1 padding.  Query t scores the candidates s <= q_pos[t]
+ * of its group with its own q and w and takes its top k; idx as in
+ * pivot_group_index.  A list that is not ascending, holds a key outside its
+ * sequence or has a key after its padding is used up to its first bad entry
+ * and reported through the workspace status word (code 2, read with
+ * dsa_device_check).  Requires k <= n_cand <= 16384, 1 <= group <= 64.
+ */
+size_t pivot_refine_candidates_workspace(const dsa_batch* batch, int32_t k, int32_t group, int32_t n_cand);
+dsa_status pivot_refine_candidates(const dsa_batch* batch, const void* Q, const void* K, const float* W,
+                                   int32_t k, int32_t group, int32_t n_cand, const int32_t* cand,
+                                   int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------
  * HISA hierarchical indexing ("HISA: Efficient Hierarchical Indexing for
  * Fine-Grained Sparse Attention", abstract).
  * hisa_pool_keys: pooled [n_blocks, d] fp32, the mean of the keys of each

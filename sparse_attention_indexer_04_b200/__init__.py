@@ -65,6 +65,8 @@ _sig("dsa_index_topk", ctypes.c_int, _B, _P, _P, _P, _I32, _P, _P, _P, _SZ, _P)
 _sig("pivot_num_groups", _I32, _B, _I32)
 _sig("pivot_group_index_workspace", _SZ, _B, _I32, _I32, _I32, _I32)
 _sig("pivot_group_index", ctypes.c_int, _B, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _SZ, _P)
+_sig("pivot_refine_candidates_workspace", _SZ, _B, _I32, _I32, _I32)
+_sig("pivot_refine_candidates", ctypes.c_int, _B, _P, _P, _P, _I32, _I32, _I32, _P, _P, _P, _SZ, _P)
 _sig("hisa_num_blocks", _I64, _B, _I32)
 _sig("hisa_pool_keys", ctypes.c_int, _B, _P, _I32, _P, _P)
 _sig("hisa_index_workspace", _SZ, _B, _I32, _I32, _I32)
@@ -215,6 +217,21 @@ def pivot_group_index(layout: Layout, Q, K, W, k: int, group: int, n_cand: int, 
     _check(_lib.pivot_group_index(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), k, group, n_cand, mode, _ptr(idx),
                                   _ptr(cand), _ptr(ws), _bytes(ws), _stream(stream)), "pivot_group_index")
     return (idx, cand) if want_cand else idx
+
+
+def pivot_refine_candidates_workspace(layout: Layout, k: int, group: int, n_cand: int) -> int:
+    return int(_lib.pivot_refine_candidates_workspace(layout.ref(), k, group, n_cand))
+
+
+def pivot_refine_candidates(layout: Layout, Q, K, W, k: int, group: int, cand, idx=None, ws=None, stream=None):
+    """Refine on supplied candidates: cand [n_groups, n_cand] int32 (ascending, -1 padded) -> idx [n_q, k]."""
+    n_cand = int(cand.shape[1])
+    if idx is None:
+        idx = torch.empty(layout.num_queries, k, dtype=torch.int32, device=layout.device)
+    ws = _workspace(pivot_refine_candidates_workspace(layout, k, group, n_cand), layout.device, ws)
+    _check(_lib.pivot_refine_candidates(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), k, group, n_cand, _ptr(cand),
+                                        _ptr(idx), _ptr(ws), _bytes(ws), _stream(stream)), "pivot_refine_candidates")
+    return idx
 
 
 # -------------------------------------------------------------------- HISA

@@ -694,6 +694,22 @@ dsa_status clear_status(void* ws, cudaStream_t st)
     return cudaMemsetAsync(ws, 0, kHeaderBytes, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
+// PIVOT Refine's second stage: each query scores its eligible candidates (query_rows, list map m)
+// with its own indexer on tensor cores, the group's candidate keys gathered tile by tile.
+dsa_status refine_stage(const dsa_batch* b, const void* Q, const void* K, const float* W, int32_t k, int32_t G,
+                        int32_t C, int32_t ng, const ColMap& m, int32_t* idx, const PivotPlan& p, void* ws,
+                        cudaStream_t st)
+{
+    DSA_LAUNCH(kProfSetup, st, group_row_offsets_kernel<<<(ng + 256) / 256, 256, 0, st>>>(p.groups, ng, b->num_queries,
+                                                                                          p.group_rows));
+    dsa_status s;
+    if ((s = launched()) != DSA_OK) return s;
+    const std::vector<int32_t> groff = group_rows_host(b, G);
+    const TcSource srf{Q, b->num_queries, W, p.group_rows, groff.data(), ng};
+    return tc_score_and_select(p.query_rows, b->num_queries, srf, b->num_heads, b->head_dim, K, b->num_keys,
+                               b->k_offsets, m, C, p.S, p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k,
+                               nullptr, st);
+}
 
 }  // namespace
 
@@ -835,7 +851,8 @@ dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, c
                             p.tile_base, static_cast<uint32_t*>(ws), C, cand, C, p.cand_score, st);
     if (s != DSA_OK) return s;
     DSA_LAUNCH(kProfSetup, st, pivot_query_rows_kernel<<<(b->num_queries + 255) / 256, 256, 0, st>>>(
-        b->q_offsets, b->k_offsets, b->q_pos, b->num_seqs, b->num_queries, G, p.group_base, cand, C, p.query_rows));
+        b->q_offsets, b->k_offsets, b->q_pos, b->num_seqs, b->num_queries, G, p.group_base, cand, C, nullptr,
+        p.query_rows));
     if ((s = launched()) != DSA_OK) return s;
     ColMap m{};
     m.kind = kMapList;
@@ -861,15 +878,48 @@ dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, c
         return launch_select(p.fb_rows, b->num_queries, C, k, m, p.cand_score, C, true, idx, k, nullptr, 0, st,
                              SelectSplit{}, reuse_fallback_count(ws));
     }
-    // Refine: each query scores its eligible candidates with its own indexer (tensor cores,
-    // the group's candidate keys gathered tile by tile).
-    DSA_LAUNCH(kProfSetup, st, group_row_offsets_kernel<<<(ng + 256) / 256, 256, 0, st>>>(p.groups, ng, b->num_queries,
-                                                                                          p.group_rows));
+    return refine_stage(b, Q, K, W, k, G, C, ng, m, idx, p, ws, st);
+}
+
+size_t pivot_refine_candidates_workspace(const dsa_batch* b, int32_t k, int32_t G, int32_t C)
+{
+    return pivot_group_index_workspace(b, k, G, C, 1);
+}
+
+dsa_status pivot_refine_candidates(const dsa_batch* b, const void* Q, const void* K, const float* W, int32_t k,
+                                   int32_t G, int32_t C, const int32_t* cand, int32_t* idx, void* ws,
+                                   size_t ws_bytes, void* stream)
+{
+    HostInfo hi;
+    dsa_status s = check_batch(b, &hi);
+    if (s != DSA_OK) return s;
+    if (!pivot_args_ok(k, G, C, 1) || !select_fits(k, C)) return DSA_ERR_UNSUPPORTED;
+    if ((s = check_tensors(b, Q, K, W)) != DSA_OK) return s;
+    if (b->num_queries > 0 && (!idx || !cand)) return DSA_ERR_INVALID_ARG;
+    PivotPlan p;
+    if ((s = check_ws(ws, ws_bytes, pivot_plan(nullptr, b, hi, k, G, C, 1, &p))) != DSA_OK) return s;
+    pivot_plan(static_cast<char*>(ws), b, hi, k, G, C, 1, &p);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = clear_status(ws, st)) != DSA_OK) return s;
+    const int32_t ng = count_groups(b, G);
+    if (ng == 0) return DSA_OK;
+    DSA_LAUNCH(kProfSetup, st, pivot_groups_kernel<<<1, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos, b->num_seqs, G,
+                                                                       ng, p.group_base, p.groups, p.proxy_rows));
     if ((s = launched()) != DSA_OK) return s;
-    const std::vector<int32_t> groff = group_rows_host(b, G);
-    const TcSource srf{Q, b->num_queries, W, p.group_rows, groff.data(), ng};
-    return tc_score_and_select(p.query_rows, b->num_queries, srf, H, D, K, b->num_keys, b->k_offsets, m, C, p.S,
-                               p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, nullptr, st);
+    // the caller's lists: usable lengths (the proxy row array is free scratch here)
+    int32_t* cand_len = reinterpret_cast<int32_t*>(p.proxy_rows);
+    DSA_LAUNCH(kProfSetup, st, pivot_check_cand_kernel<<<(ng + 7) / 8, 256, 0, st>>>(cand, C, p.groups, ng, b->k_offsets,
+                                                                                      cand_len, static_cast<uint32_t*>(ws)));
+    if ((s = launched()) != DSA_OK) return s;
+    DSA_LAUNCH(kProfSetup, st, pivot_query_rows_kernel<<<(b->num_queries + 255) / 256, 256, 0, st>>>(
+        b->q_offsets, b->k_offsets, b->q_pos, b->num_seqs, b->num_queries, G, p.group_base, cand, C, cand_len,
+        p.query_rows));
+    if ((s = launched()) != DSA_OK) return s;
+    ColMap m{};
+    m.kind = kMapList;
+    m.list = cand;
+    m.list_ld = C;
+    return refine_stage(b, Q, K, W, k, G, C, ng, m, idx, p, ws, st);
 }
 
 // ------------------------------------------------------------------- HISA

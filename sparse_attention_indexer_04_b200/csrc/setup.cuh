@@ -109,9 +109,10 @@ __global__ void pivot_proxy_kernel(const GroupDesc* groups, const __nv_bfloat16*
 // One row per query for Reuse / Refine: the group's candidates (ascending,
 // -1 padded) that lie inside the query's own prefix form a prefix of the
 // candidate list; RowDesc.list = group.
+// cand_len (nullable): usable length of each group's list (entries past it are ignored).
 __global__ void pivot_query_rows_kernel(const int32_t* q_off, const int32_t* k_off, const int32_t* q_pos,
                                         int32_t n_seqs, int32_t n_q, int32_t G, const int32_t* group_base,
-                                        const int32_t* cand, int32_t C, RowDesc* rows)
+                                        const int32_t* cand, int32_t C, const int32_t* cand_len, RowDesc* rows)
 {
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= n_q) return;
@@ -119,13 +120,40 @@ __global__ void pivot_query_rows_kernel(const int32_t* q_off, const int32_t* k_o
     const int g = group_base[b] + (t - q_off[b]) / G;
     const int lim = eligible_count(q_pos[t], k_off[b + 1] - k_off[b]);   // keys s < lim
     const int32_t* c = cand + (int64_t)g * C;
-    int lo = 0, hi = C;   // first position whose candidate is >= lim or -1
+    int lo = 0, hi = cand_len ? cand_len[g] : C;   // first position whose candidate is >= lim or -1
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
         const int32_t s = c[mid];
         if (s >= 0 && s < lim) lo = mid + 1; else hi = mid;
     }
     rows[t] = RowDesc{t, b, lo, g};
+}
+
+// Checks caller-supplied candidate lists (one warp per group): strictly ascending key indices of
+// the group's sequence, then -1 padding.  len[g] = the usable prefix (up to the first -1 or the
+// first bad entry); a bad entry records kErrBadRow with detail g.
+__global__ void pivot_check_cand_kernel(const int32_t* cand, int32_t C, const GroupDesc* groups, int32_t n_groups,
+                                        const int32_t* k_off, int32_t* len, uint32_t* status)
+{
+    const int g = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (g >= n_groups) return;
+    const int seq = groups[g].seq;
+    const int L = k_off[seq + 1] - k_off[seq];
+    const int32_t* c = cand + (int64_t)g * C;
+    int first_end = C, first_bad = C;
+    for (int i = lane; i < C; i += 32) {
+        const int32_t v = c[i];
+        const int32_t prev = i > 0 ? c[i - 1] : -1;
+        if (v < 0) { first_end = min(first_end, i); continue; }
+        // a key outside the sequence, not above its predecessor, or after the padding
+        if (v >= L || (i > 0 && (prev < 0 || prev >= v))) first_bad = min(first_bad, i);
+    }
+    first_end = __reduce_min_sync(0xffffffffu, first_end);
+    first_bad = __reduce_min_sync(0xffffffffu, first_bad);
+    if (lane == 0) {
+        if (first_bad < C) record_error(status, kErrBadRow, (uint32_t)g);
+        len[g] = min(first_end, first_bad);
+    }
 }
 
 // ------------------------------------------------------------------- HISA

@@ -68,6 +68,62 @@ def test_pivot_random_positions_exact(mode):
     check_exact_sets(idx, (ref["reuse_idx"] if mode == 0 else ref["refine_idx"])[group_rows(b, G)], "idx")
 
 
+def _random_candidates(b, G, C, seed, bad_group=None):
+    """Per group: a sorted random subset of its sequence's keys (some past its queries' positions), -1
+    padded; with bad_group, that group's list has a descending pair in the middle."""
+    rng = np.random.default_rng(seed)
+    qo, ko = b.q_offsets.tolist(), b.k_offsets.tolist()
+    rows = []
+    for s in range(b.num_seqs):
+        L = ko[s + 1] - ko[s]
+        for _ in range((qo[s + 1] - qo[s] + G - 1) // G):
+            n = int(rng.integers(0, min(C, L) + 1))
+            row = np.full(C, -1, np.int32)
+            row[:n] = np.sort(rng.choice(L, size=n, replace=False))
+            rows.append(row)
+    cand = np.stack(rows)
+    if bad_group is not None:
+        n = int((cand[bad_group] >= 0).sum())
+        assert n >= 4
+        cand[bad_group, n // 2], cand[bad_group, n // 2 + 1] = cand[bad_group, n // 2 + 1], cand[bad_group, n // 2]
+    return cand
+
+
+@pytest.mark.parametrize("seed,q_lens,k_lens,mode", [(50, [64], [64], "suffix"), (51, [24, 40], [300, 90], "random")])
+def test_refine_on_supplied_candidates_exact(seed, q_lens, k_lens, mode):
+    """Refine over the caller's candidate lists equals the oracle's Refine on the same lists (integer,
+    exact), including queries with no eligible candidate."""
+    import sparse_attention_indexer_04_b200 as dsa
+    import torch
+    b = workloads.ragged(seed, q_lens, k_lens, H=4, d=32, k=16, integer=True, pos_mode=mode)
+    G, C, k = 8, 48, 16
+    cand = _random_candidates(b, G, C, seed)
+    d = Dev(b)
+    ws = torch.empty(dsa.pivot_refine_candidates_workspace(d.lay, k, G, C), dtype=torch.uint8, device="cuda:0")
+    idx = dsa.pivot_refine_candidates(d.lay, d.Q, d.K, d.W, k, G, torch.as_tensor(cand).cuda(), ws=ws)
+    assert dsa.device_check(ws) == 0
+    ref = oracle.pivot(b, G, C, k, ext_cand=cand)
+    check_exact_sets(idx.cpu().numpy(), ref["refine_idx"][group_rows(b, G)], "idx")
+
+
+def test_refine_on_supplied_candidates_reports_a_bad_list():
+    """A list with a descending pair is used up to it and reported (status code 2); other groups are exact."""
+    import sparse_attention_indexer_04_b200 as dsa
+    import torch
+    b = workloads.tiny_integer(seed=52, T=256, H=4, d=32, k=16)
+    G, C, k = 8, 64, 16
+    cand = _random_candidates(b, G, C, 52, bad_group=5)
+    d = Dev(b)
+    ws = torch.empty(dsa.pivot_refine_candidates_workspace(d.lay, k, G, C), dtype=torch.uint8, device="cuda:0")
+    idx = dsa.pivot_refine_candidates(d.lay, d.Q, d.K, d.W, k, G, torch.as_tensor(cand).cuda(), ws=ws).cpu().numpy()
+    assert dsa.device_check(ws) == 2
+    good = cand.copy()
+    n = int((good[5] >= 0).sum())
+    good[5, n // 2 + 1:] = -1                   # the usable prefix: up to the larger of the swapped pair
+    ref = oracle.pivot(b, G, C, k, ext_cand=good)
+    check_exact_sets(idx, ref["refine_idx"][group_rows(b, G)], "idx")
+
+
 def test_pivot_reuse_long_groups_exact():
     """Reuse over a long prefill: groups of 16 consecutive queries, each query dropping up to 15 of the
     group's k + 15 best candidates; integer inputs with many ties, exact against the oracle."""
@@ -167,6 +223,16 @@ def test_hisa_integer_exact(B, keep):
     b = workloads.ragged(9, [3, 2, 4], [1500, 700, 129], H=4, d=32, k=100, integer=True, pos_mode="random")
     idx, kept, _ = Dev(b).hisa(100, B, keep)
     ref = oracle.hisa(b, B, keep, 100)
+    check_exact_sets(kept, ref["kept"], "kept")
+    check_exact_sets(idx, ref["idx"], "idx")
+
+
+def test_hisa_prefill_exact():
+    """HISA in prefill (every position of a sequence is a query: the block filter runs per query over
+    its own causal prefix); integer inputs, exact kept blocks and indices."""
+    b = workloads.tiny_integer(seed=10, T=1500, H=4, d=32, k=96)
+    idx, kept, _ = Dev(b).hisa(96, 64, 5)
+    ref = oracle.hisa(b, 64, 5, 96)
     check_exact_sets(kept, ref["kept"], "kept")
     check_exact_sets(idx, ref["idx"], "idx")
 
