@@ -82,10 +82,10 @@ def _random_candidates(b, G, C, seed, bad_group=None):
             row[:n] = np.sort(rng.choice(L, size=n, replace=False))
             rows.append(row)
     cand = np.stack(rows)
-    if bad_group is not None:
-        n = int((cand[bad_group] >= 0).sum())
-        assert n >= 4
-        cand[bad_group, n // 2], cand[bad_group, n // 2 + 1] = cand[bad_group, n // 2 + 1], cand[bad_group, n // 2]
+    if bad_group is not None:   # single-sequence batch: a 32-key list with its middle pair swapped
+        cand[bad_group] = -1
+        cand[bad_group, :32] = np.sort(rng.choice(ko[1] - ko[0], size=32, replace=False))
+        cand[bad_group, 16], cand[bad_group, 17] = cand[bad_group, 17], cand[bad_group, 16]
     return cand
 
 
@@ -118,8 +118,7 @@ def test_refine_on_supplied_candidates_reports_a_bad_list():
     idx = dsa.pivot_refine_candidates(d.lay, d.Q, d.K, d.W, k, G, torch.as_tensor(cand).cuda(), ws=ws).cpu().numpy()
     assert dsa.device_check(ws) == 2
     good = cand.copy()
-    n = int((good[5] >= 0).sum())
-    good[5, n // 2 + 1:] = -1                   # the usable prefix: up to the larger of the swapped pair
+    good[5, 17:] = -1                           # the usable prefix: up to the larger of the swapped pair
     ref = oracle.pivot(b, G, C, k, ext_cand=good)
     check_exact_sets(idx, ref["refine_idx"][group_rows(b, G)], "idx")
 
