@@ -210,7 +210,7 @@ int select_threads(int32_t n_rows, int32_t k) { return n_rows < 2 * 148 || k >= 
 // bitmaps of max_cols columns (a smaller buffer only sends more rows down the full-row path).
 int32_t select_cap(int32_t k, int32_t max_cols)
 {
-    const size_t fixed = select_smem_bytes(std::max(max_cols, 1), 0) + 2048;
+    const size_t fixed = select_smem_bytes(std::max(max_cols, 1), 0, k) + 2048;
     const int fit = (int)(((size_t)227 * 1024 - fixed) / 8) & ~255;
     return std::max(256, std::min(select_buf_cap(k), fit));
 }
@@ -219,7 +219,7 @@ int32_t select_cap(int32_t k, int32_t max_cols)
 // at least 256 entries, two column bitmaps): up to about 760,000 columns.
 bool select_fits(int32_t k, int32_t max_cols)
 {
-    return select_smem_bytes(std::max(max_cols, 1), select_cap(k, max_cols)) <= (size_t)227 * 1024;
+    return select_smem_bytes(std::max(max_cols, 1), select_cap(k, max_cols), k) <= (size_t)227 * 1024;
 }
 
 // Scratch of the split-row select: two counters per row in the workspace header (zero between
@@ -265,8 +265,8 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
     a.n_rows_dev = n_rows_dev;
     a.out_from_qrow = n_rows_dev ? 1 : 0;
     a.buf_cap = select_cap(k, max_cols);
-    a.sample_bytes = (int32_t)select_sample_bytes(std::max(max_cols, 1));
-    const size_t smem = select_smem_bytes(std::max(max_cols, 1), a.buf_cap);
+    a.sample_bytes = (int32_t)select_sample_bytes(std::max(max_cols, 1), k);
+    const size_t smem = select_smem_bytes(std::max(max_cols, 1), a.buf_cap, k);
     dsa_status s;
     const int P = select_parts(n_rows, max_cols);
     if (sp.buf && sp.ctr && n_rows <= sp.max_rows && P > 1 && !n_rows_dev) {

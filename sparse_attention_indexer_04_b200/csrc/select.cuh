@@ -5,10 +5,10 @@
 // go to the lower key index.  Columns are written in ascending order.
 //
 // A row is ranked in four steps:
-//   1. threshold: the keys of m evenly spaced columns (m = 2048 per 64K
-//      columns, at most 8192) are ranked and the one at rank k*m/n plus a
-//      4-sigma margin becomes tau (rows that fit the candidate buffer skip
-//      this and keep every column);
+//   1. threshold: the keys of m evenly spaced columns (m >= 128 n / k, 2048
+//      to 8192) are ranked and the one at rank k*m/n plus a 4-sigma margin
+//      becomes tau (rows that fit the candidate buffer skip this and keep
+//      every column);
 //   2. one streaming pass appends every column with key >= tau to a
 //      candidate buffer (about 1.75 k entries);
 //   3. if at least k columns passed and none was dropped, the top k of the
@@ -29,12 +29,14 @@ namespace dsa {
 constexpr int kSampleMin = 2048;
 constexpr int kSampleMax = 8192;
 
-// Sample size for a row of n columns: 2048 per 65536 columns, 2048 to 8192, so the expected rank of
-// the k-th largest key in the sample (k * m / n) stays at 64 or more up to n = 256K for k = 2048.
-__host__ __device__ inline int select_sample_size(int n)
+// Sample size for a row of n columns and rank k: enough that the expected rank of the k-th
+// largest key in the sample, k * m / n, is 128 or more (the candidate count then stays within
+// the 1.75 k buffer by several standard deviations), in multiples of 2048, 2048 to 8192.
+__host__ __device__ inline int select_sample_size(int n, int k)
 {
-    const int m = kSampleMin * ((n + 65535) / 65536);
-    return m < kSampleMin ? kSampleMin : (m > kSampleMax ? kSampleMax : m);
+    const int64_t need = (128 * (int64_t)n + k - 1) / (k > 0 ? k : 1);
+    const int64_t m = (need + kSampleMin - 1) / kSampleMin * kSampleMin;
+    return m < kSampleMin ? kSampleMin : (m > kSampleMax ? kSampleMax : (int)m);
 }
 
 // Candidate buffer entries for top-k: at least 4096 and 1.75 k.
@@ -53,7 +55,7 @@ struct SelectArgs {
     int64_t ld_s;
     int32_t src_from_list;   // 1: the score row is rows[r].list instead of r
     int32_t buf_cap;         // candidate buffer entries
-    int32_t sample_bytes;    // shared memory of the sample: select_sample_bytes(max_cols)
+    int32_t sample_bytes;    // shared memory of the sample: select_sample_bytes(max_cols, k)
     int32_t* out_idx;        // [n_rows, ld_idx]
     int64_t ld_idx;
     float* out_score;        // nullable, [n_rows, ld_score]
@@ -66,12 +68,15 @@ struct SelectArgs {
 
 // Dynamic shared memory of the select kernels for rows of up to max_cols columns: the sample, the
 // candidate buffer and two bitmaps of the row's columns.
-__host__ __device__ inline size_t select_sample_bytes(int max_cols) { return (size_t)select_sample_size(max_cols) * 4; }
+__host__ __device__ inline size_t select_sample_bytes(int max_cols, int k)
+{
+    return (size_t)select_sample_size(max_cols, k) * 4;
+}
 
-__host__ __device__ inline size_t select_smem_bytes(int max_cols, int buf_cap)
+__host__ __device__ inline size_t select_smem_bytes(int max_cols, int buf_cap, int k)
 {
     const size_t words = (size_t)(max_cols + 31) / 32;
-    return select_sample_bytes(max_cols) + (size_t)buf_cap * 8 + 2 * words * 4;
+    return select_sample_bytes(max_cols, k) + (size_t)buf_cap * 8 + 2 * words * 4;
 }
 
 // Exact rank selection among `count` keys given by get(i): returns the key T
@@ -168,7 +173,7 @@ struct alignas(16) SelScalars {
 };
 
 // 1. tau for a row of n > k columns: 0 (every column is a candidate) when n <= buf_cap, else
-// the key at rank expect + 4 sqrt(expect) + 4 among m = select_sample_size(n) evenly spaced
+// the key at rank expect + 4 sqrt(expect) + 4 among m = select_sample_size(n, k) evenly spaced
 // columns, expect = k * m / n (the expected rank of the k-th largest key in the sample, plus a
 // margin).
 template <int NT>
@@ -177,7 +182,7 @@ __device__ __forceinline__ uint32_t sel_threshold(const float* src, int n, int k
 {
     if (n <= buf_cap) return 0u;
     const int tid = threadIdx.x;
-    const int m = select_sample_size(n);   // a multiple of 2048
+    const int m = select_sample_size(n, k);   // a multiple of 2048
     constexpr int J = kSampleMin / NT;     // sample loads in flight per thread
     for (int j0 = 0; j0 < m; j0 += kSampleMin) {
         float x[J];
