@@ -126,6 +126,29 @@ dsa_status dsa_index_topk(const dsa_batch* batch, const void* Q, const void* K, 
                           void* stream);
 
 /* --------------------------------------------------------------------
+ * Dense top-k from host memory (no counterpart in the pages; the same
+ * computation as dsa_index_topk for inputs that live in host memory).
+ * Q, K, W, q_pos_host and idx are HOST pointers (page-locked for the copies
+ * to overlap; pageable memory works but serialises); batch->q_offsets_host
+ * and k_offsets_host are used and the batch's device pointer fields are
+ * ignored.  The rows are processed in the same chunks as dsa_index_topk:
+ * while chunk c is scored and selected on `stream`, chunk c+1's queries are
+ * copied in on `in_stream` and chunk c-1's indices copied out on
+ * `out_stream` (K, W and q_pos are copied once, first).  in_stream and
+ * out_stream must differ from `stream` (they may be the same stream, which
+ * serialises the two directions).  Returns after enqueueing; idx is
+ * complete when `stream` has passed the call's work.  The workspace
+ * (dsa_index_topk_host_workspace bytes) holds dsa_index_topk's workspace
+ * followed by device copies of K, W, q_pos, the offsets and two chunks of
+ * queries and of indices.  The status word is at the workspace start as
+ * for every call.
+ */
+size_t dsa_index_topk_host_workspace(const dsa_batch* batch, int32_t k);
+dsa_status dsa_index_topk_host(const dsa_batch* batch, const int32_t* q_pos_host, const void* Q, const void* K,
+                               const float* W, int32_t k, int32_t* idx, void* ws, size_t ws_bytes,
+                               void* stream, void* in_stream, void* out_stream);
+
+/* --------------------------------------------------------------------
  * PIVOT group-proxy indexing ("PIVOT: Efficient Query-Group Indexing for
  * Token-Level Sparse Attention", abstract).
  * Groups: inside each sequence, consecutive runs of `group` query rows (the

@@ -62,6 +62,8 @@ _sig("dsa_index_scores_workspace", _SZ, _B)
 _sig("dsa_index_scores", ctypes.c_int, _B, _P, _P, _P, _P, _I64, _P, _SZ, _P)
 _sig("dsa_index_topk_workspace", _SZ, _B, _I32)
 _sig("dsa_index_topk", ctypes.c_int, _B, _P, _P, _P, _I32, _P, _P, _P, _SZ, _P)
+_sig("dsa_index_topk_host_workspace", _SZ, _B, _I32)
+_sig("dsa_index_topk_host", ctypes.c_int, _B, _P, _P, _P, _P, _I32, _P, _P, _SZ, _P, _P, _P)
 _sig("pivot_num_groups", _I32, _B, _I32)
 _sig("pivot_group_index_workspace", _SZ, _B, _I32, _I32, _I32, _I32)
 _sig("pivot_group_index", ctypes.c_int, _B, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _SZ, _P)
@@ -178,6 +180,25 @@ def index_topk(layout: Layout, Q, K, W, k: int, idx=None, scores=None, want_scor
     _check(_lib.dsa_index_topk(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), k, _ptr(idx), _ptr(scores), _ptr(ws),
                                _bytes(ws), _stream(stream)), "dsa_index_topk")
     return (idx, scores) if want_scores else idx
+
+
+def index_topk_host_workspace(layout: Layout, k: int) -> int:
+    return int(_lib.dsa_index_topk_host_workspace(layout.ref(), k))
+
+
+def index_topk_host(layout: Layout, q_pos, Q, K, W, k: int, idx, ws, stream=None, in_stream=None, out_stream=None):
+    """dsa_index_topk on HOST tensors (pinned for overlap): Q, K, W, q_pos (CPU) in, idx [n_q, k] (CPU,
+    int32) out.  The copies run on in_stream / out_stream (torch.cuda.Stream) overlapped with the
+    work on `stream`; idx is complete once `stream` has passed the call."""
+    for t in (q_pos, Q, K, W, idx):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("index_topk_host takes contiguous host tensors")
+    if in_stream is None or out_stream is None:
+        raise ValueError("index_topk_host needs copy streams distinct from the compute stream")
+    _check(_lib.dsa_index_topk_host(layout.ref(), _ptr(q_pos), _ptr(Q), _ptr(K), _ptr(W), k, _ptr(idx), _ptr(ws),
+                                    _bytes(ws), _stream(stream), _stream(in_stream), _stream(out_stream)),
+           "dsa_index_topk_host")
+    return idx
 
 
 def index_topk_static(layout: Layout, Q, K, W, k: int, idx=None, scores=None, want_scores=False, stream=None):

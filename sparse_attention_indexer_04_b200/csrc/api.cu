@@ -545,6 +545,41 @@ size_t dense_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k,
     return c.off;
 }
 
+// Workspace of dsa_index_topk_host: dsa_index_topk's workspace first (its header stays at the
+// base), then device copies of the inputs and two row chunks' queries and indices.
+struct HostPlan {
+    int32_t* q_off;
+    int32_t* k_off;
+    int32_t* q_pos;
+    uint8_t* K;
+    float* W;
+    uint8_t* Q[2];
+    int32_t* idx[2];
+    RowDesc* rows;   // one chunk's rows, query rows relative to the chunk
+    int32_t chunk;
+};
+
+size_t host_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, DensePlan* dp, HostPlan* p)
+{
+    const size_t inner = dense_plan(base, b, hi, k, dp);
+    Carver c{base};
+    c.off = align256(inner);
+    const int32_t nq = std::max(1, b->num_queries);
+    const size_t qrow_bytes = size_t(b->num_heads) * b->head_dim * 2;
+    p->chunk = chunk_rows(nq, score_ld(hi.max_k));
+    p->q_off = c.take<int32_t>(b->num_seqs + 1);
+    p->k_off = c.take<int32_t>(b->num_seqs + 1);
+    p->q_pos = c.take<int32_t>(nq);
+    p->K = c.take<uint8_t>(size_t(std::max(1, b->num_keys)) * b->head_dim * 2);
+    p->W = c.take<float>(size_t(nq) * b->num_heads);
+    for (int i = 0; i < 2; ++i) {
+        p->Q[i] = c.take<uint8_t>(size_t(p->chunk) * qrow_bytes);
+        p->idx[i] = c.take<int32_t>(size_t(p->chunk) * k);
+    }
+    p->rows = c.take<RowDesc>(p->chunk);
+    return c.off;
+}
+
 struct PivotPlan {
     int32_t* group_base;
     GroupDesc* groups;
@@ -796,6 +831,117 @@ dsa_status dsa_index_topk(const dsa_batch* b, const void* Q, const void* K, cons
     return tc_score_and_select(p.rows, b->num_queries, src, b->num_heads, b->head_dim, K, b->num_keys, b->k_offsets,
                                ColMap{}, hi.max_k, p.S, p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, scores, st,
                                p.split);
+}
+
+// ------------------------------------------------- dense top-k from host memory
+size_t dsa_index_topk_host_workspace(const dsa_batch* b, int32_t k)
+{
+    dsa_batch d = *b;   // device pointers are the library's own copies here: any non-null stand-in
+    d.q_offsets = d.k_offsets = d.q_pos = reinterpret_cast<const int32_t*>(b->q_offsets_host);
+    HostInfo hi;
+    if (check_batch(&d, &hi) != DSA_OK || k < 1 || k > kMaxK) return 0;
+    DensePlan dp;
+    HostPlan hp;
+    return host_plan(nullptr, &d, hi, k, &dp, &hp);
+}
+
+dsa_status dsa_index_topk_host(const dsa_batch* b, const int32_t* q_pos_host, const void* Q, const void* K,
+                               const float* W, int32_t k, int32_t* idx, void* ws, size_t ws_bytes, void* stream,
+                               void* in_stream, void* out_stream)
+{
+    if (!b || !q_pos_host) return DSA_ERR_INVALID_ARG;
+    dsa_batch d = *b;
+    d.q_offsets = d.k_offsets = d.q_pos = reinterpret_cast<const int32_t*>(b->q_offsets_host);   // checked below
+    HostInfo hi;
+    dsa_status s = check_batch(&d, &hi);
+    if (s != DSA_OK) return s;
+    if (k < 1 || k > kMaxK || !select_fits(k, hi.max_k)) return DSA_ERR_UNSUPPORTED;
+    if ((s = check_tensors(&d, Q, K, W)) != DSA_OK) return s;
+    if (b->num_queries > 0 && !idx) return DSA_ERR_INVALID_ARG;
+    if (stream == in_stream || stream == out_stream) return DSA_ERR_INVALID_ARG;
+    DensePlan dp;
+    HostPlan hp;
+    if ((s = check_ws(ws, ws_bytes, host_plan(nullptr, &d, hi, k, &dp, &hp))) != DSA_OK) return s;
+    host_plan(static_cast<char*>(ws), &d, hi, k, &dp, &hp);
+    d.q_offsets = hp.q_off;
+    d.k_offsets = hp.k_off;
+    d.q_pos = hp.q_pos;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaStream_t si = static_cast<cudaStream_t>(in_stream), so = static_cast<cudaStream_t>(out_stream);
+    if ((s = clear_status(ws, st)) != DSA_OK) return s;
+    const int32_t nq = b->num_queries;
+    if (nq == 0) return DSA_OK;
+    const int H = b->num_heads, D = b->head_dim;
+    const size_t qrow_bytes = size_t(H) * D * 2;
+
+    // Events linking the streams (released once the device has passed them).
+    constexpr int kEvents = 9;
+    cudaEvent_t ev[kEvents];
+    int made = 0;
+    for (; made < kEvents; ++made)
+        if (cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming) != cudaSuccess) break;
+    auto release = [&]() { for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]); };
+    if (made < kEvents) { release(); return DSA_ERR_CUDA; }
+    cudaEvent_t e_start = ev[0], e_in = ev[1], e_out = ev[2];
+    cudaEvent_t e_q[2] = {ev[3], ev[4]}, e_done[2] = {ev[5], ev[6]}, e_back[2] = {ev[7], ev[8]};
+    bool ok = true;
+    auto chk = [&](cudaError_t e) { ok = ok && e == cudaSuccess; };
+    const int32_t n_chunks = (nq + hp.chunk - 1) / hp.chunk;
+    auto rows_of = [&](int32_t c) { return std::min(hp.chunk, nq - c * hp.chunk); };
+    // query rows of chunk c into buffer c % 2, once chunk c - 2 no longer reads it
+    auto send_queries = [&](int32_t c) {
+        if (c >= 2) chk(cudaStreamWaitEvent(si, e_done[c & 1], 0));
+        chk(cudaMemcpyAsync(hp.Q[c & 1], static_cast<const uint8_t*>(Q) + size_t(c) * hp.chunk * qrow_bytes,
+                            size_t(rows_of(c)) * qrow_bytes, cudaMemcpyHostToDevice, si));
+        chk(cudaEventRecord(e_q[c & 1], si));
+    };
+
+    // The small inputs and the keys first (after the header is cleared), then chunk 0's queries.
+    chk(cudaEventRecord(e_start, st));
+    chk(cudaStreamWaitEvent(si, e_start, 0));
+    chk(cudaStreamWaitEvent(so, e_start, 0));
+    chk(cudaMemcpyAsync(hp.q_off, b->q_offsets_host, (b->num_seqs + 1) * sizeof(int32_t), cudaMemcpyHostToDevice, si));
+    chk(cudaMemcpyAsync(hp.k_off, b->k_offsets_host, (b->num_seqs + 1) * sizeof(int32_t), cudaMemcpyHostToDevice, si));
+    chk(cudaMemcpyAsync(hp.q_pos, q_pos_host, size_t(nq) * sizeof(int32_t), cudaMemcpyHostToDevice, si));
+    chk(cudaMemcpyAsync(hp.W, W, size_t(nq) * H * sizeof(float), cudaMemcpyHostToDevice, si));
+    if (b->num_keys > 0) chk(cudaMemcpyAsync(hp.K, K, size_t(b->num_keys) * D * 2, cudaMemcpyHostToDevice, si));
+    chk(cudaEventRecord(e_in, si));
+    send_queries(0);
+    chk(cudaStreamWaitEvent(st, e_in, 0));
+    if (!ok) { release(); return DSA_ERR_CUDA; }
+    DSA_LAUNCH(kProfSetup, st, dense_rows_kernel<<<(nq + 255) / 256, 256, 0, st>>>(d.q_offsets, d.k_offsets, d.q_pos,
+                                                                                  d.num_seqs, nq, dp.rows));
+    if ((s = launched()) != DSA_OK) { release(); return s; }
+
+    // Row chunks: while chunk c is scored and selected, chunk c+1's queries come in and chunk c-1's
+    // indices go out.
+    const int64_t ld = score_ld(hi.max_k);
+    for (int32_t c = 0; c < n_chunks && ok; ++c) {
+        const int32_t r0 = c * hp.chunk, nr = rows_of(c);
+        const int x = c & 1;
+        chk(cudaStreamWaitEvent(st, e_q[x], 0));
+        if (c >= 2) chk(cudaStreamWaitEvent(st, e_back[x], 0));   // chunk c-2's indices have left idx[x]
+        DSA_LAUNCH(kProfSetup, st, chunk_rows_kernel<<<(nr + 255) / 256, 256, 0, st>>>(dp.rows, r0, nr, hp.rows));
+        if ((s = launched()) != DSA_OK) break;
+        const TcSource src{hp.Q[x], nr, hp.W + size_t(r0) * H, d.q_offsets, b->q_offsets_host, b->num_seqs};
+        s = tc_score(hp.rows, nr, r0, src, H, D, hp.K, b->num_keys, d.k_offsets, ColMap{}, hi.max_k, dp.S, ld, dp.units,
+                     dp.tile_base, static_cast<uint32_t*>(ws), st);
+        if (s != DSA_OK) break;
+        s = launch_select(hp.rows, nr, hi.max_k, k, ColMap{}, dp.S, ld, false, hp.idx[x], k, nullptr, 0, st, dp.split);
+        if (s != DSA_OK) break;
+        chk(cudaEventRecord(e_done[x], st));
+        if (c + 1 < n_chunks) send_queries(c + 1);
+        chk(cudaStreamWaitEvent(so, e_done[x], 0));
+        chk(cudaMemcpyAsync(idx + size_t(r0) * k, hp.idx[x], size_t(nr) * k * sizeof(int32_t), cudaMemcpyDeviceToHost,
+                            so));
+        chk(cudaEventRecord(e_back[x], so));
+    }
+    // The caller's stream completes after the last index copy.
+    chk(cudaEventRecord(e_out, so));
+    chk(cudaStreamWaitEvent(st, e_out, 0));
+    release();
+    if (s != DSA_OK) return s;
+    return ok ? DSA_OK : DSA_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ PIVOT

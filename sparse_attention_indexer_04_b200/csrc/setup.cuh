@@ -19,6 +19,17 @@ __global__ void dense_rows_kernel(const int32_t* q_off, const int32_t* k_off, co
     rows[t] = RowDesc{t, b, eligible_count(q_pos[t], k_off[b + 1] - k_off[b]), 0};
 }
 
+// Rows [r0, r0 + n) of a row array, with their query rows made relative to r0 (a row chunk whose
+// queries sit in a buffer of their own).
+__global__ void chunk_rows_kernel(const RowDesc* rows, int32_t r0, int32_t n, RowDesc* out)
+{
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= n) return;
+    RowDesc r = rows[r0 + j];
+    r.qrow -= r0;
+    out[j] = r;
+}
+
 // ------------------------------------------------------------------ PIVOT
 // PIVOT ("PIVOT: Efficient Query-Group Indexing for Token-Level Sparse
 // Attention", abstract): inside each sequence, consecutive runs of G query

@@ -100,6 +100,19 @@ def test_argument_errors_return_before_any_launch():
     assert call_topk(host_layout([1], [1_000_000]), k=2048) == 2
 
 
+def test_host_entry_argument_errors_need_no_gpu():
+    lib = dsa.library()
+    lay = host_layout([8], [8])
+    P = ctypes.c_void_p
+    args = lambda **kw: [lay.ref(), P(kw.get("pos", 0x800)), P(0x1000), P(0x2000), P(0x3000), kw.get("k", 4),
+                         P(0x4000), P(0x10000), ctypes.c_size_t(1 << 30), P(kw.get("st", 0)), P(kw.get("si", 1)),
+                         P(kw.get("so", 2))]
+    assert lib.dsa_index_topk_host(*args(pos=0)) == 1          # missing positions
+    assert lib.dsa_index_topk_host(*args(k=0)) == 2            # unsupported k
+    assert lib.dsa_index_topk_host(*args(si=0)) == 1           # copy stream = compute stream
+    assert lib.dsa_index_topk_host_workspace(lay.ref(), 4) > lib.dsa_index_topk_workspace(lay.ref(), 4)
+
+
 def test_selftest_argument_errors_need_no_gpu():
     lib = dsa.library()
     P = ctypes.c_void_p

@@ -161,3 +161,26 @@ def test_few_long_rows_exact(seed, q_lens, k_lens, k, mode):
     buffer.  Integer inputs (many ties across the CTAs' column chunks), a row shorter than k, clamped
     positions; exact against the oracle."""
     exact_topk(workloads.ragged(seed, q_lens, k_lens, H=4, d=32, k=k, integer=True, pos_mode=mode), k)
+
+
+@pytest.mark.parametrize("make", [
+    lambda: workloads.dense_prefill(seed=2),                                     # 4 row chunks, pipelined
+    lambda: workloads.ragged(60, [5, 0, 64], [300, 17, 129], H=4, d=32, k=24),   # one chunk, ragged
+    lambda: workloads.dense_decode(seed=61, B=4, L=5000, n_mtp=2, H=64, d=128, k=256),
+])
+def test_host_memory_entry_matches_device_entry(make):
+    """dsa_index_topk_host (inputs and indices in pinned host memory, copies overlapped with the work)
+    returns exactly what dsa_index_topk returns on device copies of the same inputs."""
+    import sparse_attention_indexer_04_b200 as dsa
+    b = make()
+    k = int(b.params["k"])
+    d = Dev(b)
+    ref = d.topk(k)
+    hidx = torch.full((b.n_q, k), -7, dtype=torch.int32).pin_memory()
+    ws = torch.empty(dsa.index_topk_host_workspace(d.lay, k), dtype=torch.uint8, device="cuda:0")
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    dsa.index_topk_host(d.lay, b.q_pos.to(torch.int32).contiguous().pin_memory(), b.Q.pin_memory(), b.K.pin_memory(),
+                        b.W.contiguous().pin_memory(), k, hidx, ws, in_stream=s_in, out_stream=s_out)
+    torch.cuda.current_stream().synchronize()
+    assert dsa.device_check(ws) == 0
+    assert np.array_equal(hidx.numpy(), ref)
