@@ -5,10 +5,10 @@
 // go to the lower key index.  Columns are written in ascending order.
 //
 // A row is ranked in four steps:
-//   1. threshold: the keys of m evenly spaced columns (m >= 128 n / k, 2048
-//      to 8192) are ranked and the one at rank k*m/n plus a 4-sigma margin
-//      becomes tau (rows that fit the candidate buffer skip this and keep
-//      every column);
+//   1. threshold: the keys of m columns (m >= 128 n / k, 2048 to 8192), in
+//      m/32 evenly spaced runs of 32, are ranked and the one at rank k*m/n
+//      plus a 4-sigma margin becomes tau (rows that fit the candidate buffer
+//      skip this and keep every column);
 //   2. one streaming pass appends every column with key >= tau to a
 //      candidate buffer (about 1.75 k entries);
 //   3. if at least k columns passed and none was dropped, the top k of the
@@ -173,7 +173,7 @@ struct alignas(16) SelScalars {
 };
 
 // 1. tau for a row of n > k columns: 0 (every column is a candidate) when n <= buf_cap, else
-// the key at rank expect + 4 sqrt(expect) + 4 among m = select_sample_size(n, k) evenly spaced
+// the key at rank expect + 4 sqrt(expect) + 4 among m = select_sample_size(n, k) sampled
 // columns, expect = k * m / n (the expected rank of the k-th largest key in the sample, plus a
 // margin).
 template <int NT>
@@ -183,11 +183,19 @@ __device__ __forceinline__ uint32_t sel_threshold(const float* src, int n, int k
     if (n <= buf_cap) return 0u;
     const int tid = threadIdx.x;
     const int m = select_sample_size(n, k);   // a multiple of 2048
+    // m / 32 evenly spaced runs of 32 consecutive columns (a warp reads one run: one or two cache
+    // lines instead of 32 scattered sectors); run r starts at floor(r n / R) rounded down to 32.
+    const int R = m / 32;
     constexpr int J = kSampleMin / NT;     // sample loads in flight per thread
     for (int j0 = 0; j0 < m; j0 += kSampleMin) {
         float x[J];
 #pragma unroll
-        for (int j = 0; j < J; ++j) x[j] = __ldg(src + (int)(((int64_t)(j0 + tid + j * NT) * n) / m));
+        for (int j = 0; j < J; ++j) {
+            const int sidx = j0 + tid + j * NT;
+            const int run = sidx >> 5;
+            const int col = (int)((((int64_t)run * n / R) & ~31ll) + (sidx & 31));
+            x[j] = __ldg(src + min(col, n - 1));   // runs narrower than 32 columns (n < 32 R) stop at the row's end
+        }
 #pragma unroll
         for (int j = 0; j < J; ++j) sample[j0 + tid + j * NT] = score_key(x[j]);
     }

@@ -131,13 +131,14 @@ def test_full_size_prefill_32k_sampled_rows():
 @pytest.mark.parametrize("n_rows", [2, 300])
 @pytest.mark.parametrize("sampled_high", [True, False])
 def test_select_when_the_even_sample_misleads(sampled_high, n_rows):
-    """The top-k picks a threshold from 2048 evenly spaced columns of a long row.  Keys that make exactly
-    those columns score high (too few columns then pass the threshold) or low (too many pass) must still
-    give the exact answer: integer inputs, compared exactly with the oracle.  Two rows take the split
-    select (several CTAs per row), 300 rows the one-CTA-per-row select."""
+    """The top-k picks a threshold from a sample of a long row: 2048 columns in 64 evenly spaced runs of
+    32.  Keys that make exactly those columns score high (too few columns then pass the threshold) or
+    low (too many pass) must still give the exact answer: integer inputs, compared exactly with the
+    oracle.  Two rows take the split select (several CTAs per row), 300 rows the one-CTA-per-row select."""
     L, k = 20000, 3000
     b = workloads.ragged(30, [n_rows], [L], H=1, d=32, k=k, integer=True)
-    sampled = np.unique((np.arange(2048, dtype=np.int64) * L) // 2048)    # the sample of a row of n = L
+    starts = ((np.arange(64, dtype=np.int64) * L) // 64) & ~31        # the sample of a row of n = L
+    sampled = np.unique((starts[:, None] + np.arange(32)[None, :]).ravel())
     hi, lo = (3.0, 1.0) if sampled_high else (1.0, 3.0)
     K = np.full((L, 32), lo, np.float32)
     K[sampled] = hi
