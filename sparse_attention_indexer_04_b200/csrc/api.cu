@@ -26,7 +26,7 @@ constexpr int32_t kMaxCand = 16384;
 // Bytes of materialised score rows per launch: 1 GiB keeps a 32K prefill's scoring launches at
 // ~1000 units (about 7 waves of 148 SMs), where 256 MiB (256 units, 1.7 waves) lost ~14 % to
 // the last wave.
-constexpr size_t kScoreBudget = size_t(1024) << 20;   // bytes of materialised score rows per launch
+constexpr size_t kScoreBudget = size_t(1024) << 20;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
