@@ -101,14 +101,25 @@ __global__ void pivot_proxy_kernel(const GroupDesc* groups, const __nv_bfloat16*
                                    int32_t H, int32_t D, __nv_bfloat16* Qp, float* Wp)
 {
     const GroupDesc g = groups[blockIdx.x];
-    const int HD = H * D;
-    const uint16_t* q = reinterpret_cast<const uint16_t*>(Q);
-    uint16_t* qp = reinterpret_cast<uint16_t*>(Qp) + (int64_t)blockIdx.x * HD;
-    for (int e = threadIdx.x; e < HD; e += blockDim.x) {
-        double s = 0.0;
-        for (int j = 0; j < g.size; ++j)
-            s += (double)__uint_as_float((uint32_t)q[(int64_t)(g.first + j) * HD + e] << 16);
-        qp[e] = bf16_bits_rne(s / g.size);
+    const int HD8 = H * D / 8;   // 16-byte groups of 8 elements per query row (D >= 32)
+    const uint4* q = reinterpret_cast<const uint4*>(Q);
+    uint4* qp = reinterpret_cast<uint4*>(Qp) + (int64_t)blockIdx.x * HD8;
+    for (int e8 = threadIdx.x; e8 < HD8; e8 += blockDim.x) {
+        double s[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};   // summed in query order
+        for (int j = 0; j < g.size; ++j) {
+            const uint4 v = __ldg(q + (int64_t)(g.first + j) * HD8 + e8);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                s[2 * e] += (double)__uint_as_float(w[e] << 16);                 // low half: element 2e
+                s[2 * e + 1] += (double)__uint_as_float(w[e] & 0xffff0000u);    // high half: element 2e+1
+            }
+        }
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            o[e] = (uint32_t)bf16_bits_rne(s[2 * e] / g.size) | ((uint32_t)bf16_bits_rne(s[2 * e + 1] / g.size) << 16);
+        qp[e8] = make_uint4(o[0], o[1], o[2], o[3]);
     }
     for (int h = threadIdx.x; h < H; h += blockDim.x) {
         double s = 0.0;
