@@ -89,19 +89,13 @@ __host__ __device__ inline size_t select_smem_bytes(int max_cols, int buf_cap, i
 // taken).  With stop_bits > 0 only the top stop_bits bits of (key - min) are
 // resolved and the lower edge of that bin is returned: a key <= T (krem is
 // then meaningless).  All threads call it.
-template <int NT, typename Get>
-__device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, uint32_t* hist, uint32_t* scratch,
-                                                 int stop_bits = 0)
+// Block-wide min and max of the keys each thread passes in (lo, hi): every thread gets the result.
+// Ends with a barrier, so shared-memory writes made before the call are visible after it.
+template <int NT>
+__device__ __forceinline__ void block_key_range(uint32_t& lo, uint32_t& hi, uint32_t* scratch)
 {
-    constexpr int kSelThreads = NT;
     constexpr int kSelWarps = NT / 32;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t lo = 0xffffffffu, hi = 0u;
-    for (int i = tid; i < count; i += kSelThreads) {
-        const uint32_t u = get(i);
-        lo = min(lo, u);
-        hi = max(hi, u);
-    }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     lo = __reduce_min_sync(0xffffffffu, lo);
     hi = __reduce_max_sync(0xffffffffu, hi);
     __syncthreads();
@@ -111,6 +105,16 @@ __device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, 
     hi = scratch[kSelWarps];
 #pragma unroll
     for (int w = 1; w < kSelWarps; ++w) { lo = min(lo, scratch[w]); hi = max(hi, scratch[kSelWarps + w]); }
+}
+
+// radix_select with the keys' block-wide range [lo, hi] already known (all threads pass the same).
+template <int NT, typename Get>
+__device__ __forceinline__ uint32_t radix_select_in(Get get, int count, int& krem, uint32_t lo, uint32_t hi,
+                                                    uint32_t* hist, uint32_t* scratch, int stop_bits = 0)
+{
+    constexpr int kSelThreads = NT;
+    constexpr int kSelWarps = NT / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int top = 32 - __clz(hi - lo);   // bits of (key - lo) still undecided
     const int stop = stop_bits > 0 ? max(top - stop_bits, 0) : 0;
     uint32_t prefix = 0;             // decided high bits of (T - lo)
@@ -121,7 +125,7 @@ __device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, 
         __syncthreads();
         for (int i = tid; i < count; i += kSelThreads) {
             const uint32_t rel = get(i) - lo;
-            if ((uint32_t)((uint64_t)rel >> top) == prefix) atomicAdd(&hist[(rel >> shift) & ((1u << width) - 1u)], 1u);
+            if (((rel >> 1) >> (top - 1)) == prefix) atomicAdd(&hist[(rel >> shift) & ((1u << width) - 1u)], 1u);
         }
         __syncthreads();
         if (warp == 0) {
@@ -162,6 +166,20 @@ __device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, 
     return lo + (prefix << top);
 }
 
+template <int NT, typename Get>
+__device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, uint32_t* hist, uint32_t* scratch,
+                                                 int stop_bits = 0)
+{
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int i = threadIdx.x; i < count; i += NT) {
+        const uint32_t u = get(i);
+        lo = min(lo, u);
+        hi = max(hi, u);
+    }
+    block_key_range<NT>(lo, hi, scratch);
+    return radix_select_in<NT>(get, count, krem, lo, hi, hist, scratch, stop_bits);
+}
+
 // Shared scalars of one selection CTA.
 template <int NT>
 struct alignas(16) SelScalars {
@@ -181,30 +199,39 @@ __device__ __forceinline__ uint32_t sel_threshold(const float* src, int n, int k
                                                   SelScalars<NT>& sh)
 {
     if (n <= buf_cap) return 0u;
-    const int tid = threadIdx.x;
+    static_assert(NT >= 256 && kSampleMax / NT <= 32, "one run start per lane");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int m = select_sample_size(n, k);   // a multiple of 2048
     // m / 32 evenly spaced runs of 32 consecutive columns (a warp reads one run: one or two cache
     // lines instead of 32 scattered sectors); run r starts at floor(r n / R) rounded down to 32.
-    const int R = m / 32;
+    // Sample entry e belongs to run e / 32, so a warp's i-th run is warp + i NT / 32; lane i
+    // computes that run's start once (r n < 2^31: 32-bit arithmetic) and the loads fetch it by shuffle.
+    const uint32_t R = (uint32_t)(m / 32);
+    const uint32_t my_run = (uint32_t)(warp + lane * (NT / 32));
+    const int my_start = my_run < R ? (int)(((my_run * (uint32_t)n) / R) & ~31u) : 0;
     constexpr int J = kSampleMin / NT;     // sample loads in flight per thread
+    uint32_t lo = 0xffffffffu, hi = 0u;
     for (int j0 = 0; j0 < m; j0 += kSampleMin) {
         float x[J];
 #pragma unroll
         for (int j = 0; j < J; ++j) {
-            const int sidx = j0 + tid + j * NT;
-            const int run = sidx >> 5;
-            const int col = (int)((((int64_t)run * n / R) & ~31ll) + (sidx & 31));
+            const int col = __shfl_sync(0xffffffffu, my_start, j0 / NT + j) + lane;
             x[j] = __ldg(src + min(col, n - 1));   // runs narrower than 32 columns (n < 32 R) stop at the row's end
         }
 #pragma unroll
-        for (int j = 0; j < J; ++j) sample[j0 + tid + j * NT] = score_key(x[j]);
+        for (int j = 0; j < J; ++j) {
+            const uint32_t u = score_key(x[j]);
+            sample[j0 + tid + j * NT] = u;
+            lo = min(lo, u);
+            hi = max(hi, u);
+        }
     }
     const float expect = (float)k * m / n;
     int rank = (int)ceilf(expect + 4.f * sqrtf(expect) + 4.f);
     rank = min(rank, m);
-    __syncthreads();
+    block_key_range<NT>(lo, hi, sh.scratch);   // its barriers also publish the sample
     // 16 bits of the sample's key range are enough: the bin's lower edge only lowers tau a little
-    return radix_select<NT>([&](int i) { return sample[i]; }, m, rank, sh.hist, sh.scratch, 16);
+    return radix_select_in<NT>([&](int i) { return sample[i]; }, m, rank, lo, hi, sh.hist, sh.scratch, 16);
 }
 
 // 2. Appends (key << 32 | column) of every column c in [c0, c1) whose key is >= tau to buf, one
@@ -303,16 +330,20 @@ __device__ __forceinline__ void sel_mark_all(int n, uint32_t* gtmap)
 
 // 4. Emits the marked columns in column order (all of gtmap, the first krem of eqmap), then pads
 // the row to k with -1 (and NaN scores).  Thread t owns a contiguous run of bitmap words; one
-// block-wide scan of its (> T, == T) counts gives both its output offset and its tie rank.
+// block-wide scan of its (> T, == T) counts gives both its output offset and its tie rank.  When
+// the row fits in stage (16-byte aligned, stage_words words: k, or 2k with scores) it is assembled
+// there and written with coalesced 16-byte stores, else written directly.
 template <int NT>
 __device__ __forceinline__ void sel_emit(const SelectArgs& a, const RowDesc& rd, int r, const float* src, int n,
-                                         int krem, const uint32_t* gtmap, const uint32_t* eqmap, SelScalars<NT>& sh)
+                                         int krem, const uint32_t* gtmap, const uint32_t* eqmap, int32_t* stage,
+                                         int stage_words, SelScalars<NT>& sh)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int k = a.k;
     const int nwords = (n + 31) >> 5;
     int32_t* oidx = a.out_idx + (int64_t)r * a.ld_idx;
     float* osc = a.out_score ? a.out_score + (int64_t)r * a.ld_score : nullptr;
+    const bool staged = (osc ? 2 * k : k) <= stage_words;
     const int wpt = (nwords + NT - 1) / NT;
     const int w0 = min(nwords, tid * wpt), w1 = min(nwords, w0 + wpt);
     uint32_t ng = 0, ne = 0;
@@ -343,15 +374,55 @@ __device__ __forceinline__ void sel_emit(const SelectArgs& a, const RowDesc& rd,
         }
         for (uint32_t bits = gtmap[w] | te; bits; bits &= bits - 1) {
             const int col = w * 32 + __ffs(bits) - 1;
-            oidx[out] = map_col(a.map, rd, col);
-            if (osc) osc[out] = key_score(score_key(__ldg(src + col)));
+            const int32_t key = map_col(a.map, rd, col);
+            const float sc = osc ? key_score(score_key(__ldg(src + col))) : 0.f;
+            if (staged) {
+                stage[out] = key;
+                if (osc) stage[k + out] = __float_as_int(sc);
+            } else {
+                oidx[out] = key;
+                if (osc) osc[out] = sc;
+            }
             ++out;
         }
     }
     const int n_out = min(n, k);
-    for (int j = n_out + tid; j < k; j += NT) {
-        oidx[j] = -1;
-        if (osc) osc[j] = __int_as_float(0x7fc00000);
+    constexpr int kNaN = 0x7fc00000;
+    if (!staged) {
+        for (int j = n_out + tid; j < k; j += NT) {
+            oidx[j] = -1;
+            if (osc) osc[j] = __int_as_float(kNaN);
+        }
+        return;
+    }
+    __syncthreads();
+    const bool vec = (k & 3) == 0 && ((reinterpret_cast<uintptr_t>(oidx) | reinterpret_cast<uintptr_t>(osc)) & 15) == 0;
+    if (vec) {
+        for (int j = 4 * tid; j < k; j += 4 * NT) {
+            int4 v = *reinterpret_cast<const int4*>(stage + j);
+            if (j + 3 >= n_out) {
+                v.x = j < n_out ? v.x : -1;
+                v.y = j + 1 < n_out ? v.y : -1;
+                v.z = j + 2 < n_out ? v.z : -1;
+                v.w = j + 3 < n_out ? v.w : -1;
+            }
+            *reinterpret_cast<int4*>(oidx + j) = v;
+            if (osc) {
+                int4 f = *reinterpret_cast<const int4*>(stage + k + j);
+                if (j + 3 >= n_out) {
+                    f.x = j < n_out ? f.x : kNaN;
+                    f.y = j + 1 < n_out ? f.y : kNaN;
+                    f.z = j + 2 < n_out ? f.z : kNaN;
+                    f.w = j + 3 < n_out ? f.w : kNaN;
+                }
+                *reinterpret_cast<int4*>(osc + j) = f;
+            }
+        }
+    } else {
+        for (int j = tid; j < k; j += NT) {
+            oidx[j] = j < n_out ? stage[j] : -1;
+            if (osc) osc[j] = __int_as_float(j < n_out ? stage[k + j] : kNaN);
+        }
     }
 }
 
@@ -391,7 +462,8 @@ __global__ void __launch_bounds__(NT) select_stream_kernel(SelectArgs a)
         sel_mark_all<NT>(n, gtmap);
     }
     __syncthreads();
-    sel_emit<NT>(a, rd, a.out_from_qrow ? rd.qrow : r, src, n, krem, gtmap, eqmap, sh);
+    sel_emit<NT>(a, rd, a.out_from_qrow ? rd.qrow : r, src, n, krem, gtmap, eqmap, reinterpret_cast<int32_t*>(sel_smem),
+                 (a.sample_bytes + cap * 8) / 4, sh);
 }
 
 // Few long rows: P CTAs per row (blockIdx.x = r * P + p).  Every CTA of a row derives the same
@@ -462,7 +534,8 @@ __global__ void __launch_bounds__(NT) select_split_kernel(SelectArgs a, uint64_t
         sel_mark_all<NT>(n, gtmap);
     }
     __syncthreads();
-    sel_emit<NT>(a, rd, r, src, n, krem, gtmap, eqmap, sh);
+    sel_emit<NT>(a, rd, r, src, n, krem, gtmap, eqmap, reinterpret_cast<int32_t*>(sel_smem),
+                 (a.sample_bytes + cap * 8) / 4, sh);
 }
 
 }  // namespace dsa
