@@ -234,42 +234,43 @@ __device__ __forceinline__ uint32_t sel_threshold(const float* src, int n, int k
     return radix_select_in<NT>([&](int i) { return sample[i]; }, m, rank, lo, hi, sh.hist, sh.scratch, 16);
 }
 
-// 2. Appends (key << 32 | column) of every column c in [c0, c1) whose key is >= tau to buf, one
-// shared atomic per warp and batch; sh.count (zero on entry) counts them all, entries past cap
-// are dropped.  c0 is a multiple of 4.
+// 2. Appends (key << 32 | column) of every column c in [c0, c1) whose key is >= max(tau, 1) to
+// buf; sh.count (zero on entry) counts them all, entries past cap are dropped.  (Key 0 is a NaN
+// with every bit set; leaving it out keeps the buffer exact: with k entries or more, the k-th
+// largest is >= 1.)  c0 is a multiple of 4.  Each thread loads 16 columns per round; a warp
+// finds its threads' output offsets by one prefix count over the threads' pass counts (five
+// ballots on the count's bits), takes one shared atomic, and each thread writes its passing
+// columns at consecutive slots.
 template <int NT>
 __device__ __forceinline__ void sel_append(const float* src, int c0, int c1, uint32_t tau, uint64_t* buf, int cap,
                                            SelScalars<NT>& sh)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // nv: how many of x's four columns (c .. c+3) exist.
-    auto keep4 = [&](float4 x, int c, int nv) {
-        const uint32_t u0 = score_key(x.x), u1 = score_key(x.y), u2 = score_key(x.z), u3 = score_key(x.w);
-        const bool p0 = nv > 0 && u0 >= tau, p1 = nv > 1 && u1 >= tau, p2 = nv > 2 && u2 >= tau,
-                   p3 = nv > 3 && u3 >= tau;
-        const uint32_t b0 = __ballot_sync(0xffffffffu, p0), b1 = __ballot_sync(0xffffffffu, p1);
-        const uint32_t b2 = __ballot_sync(0xffffffffu, p2), b3 = __ballot_sync(0xffffffffu, p3);
-        const uint32_t total = __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3);
-        if (total == 0) return;
+    const uint32_t t1 = max(tau, 1u);
+    const uint32_t lt = lanemask_lt();
+    // A warp's slots for `cnt` entries of this lane (cnt < 32), in lane order; returns the first.
+    auto warp_slots = [&](uint32_t cnt, uint32_t& total) {
+        uint32_t excl = 0;
+        total = 0;
+#pragma unroll
+        for (int b = 0; b < 5; ++b) {
+            const uint32_t bb = __ballot_sync(0xffffffffu, (cnt >> b) & 1u);
+            excl += __popc(bb & lt) << b;
+            total += __popc(bb) << b;
+        }
         uint32_t slot = 0;
-        if (lane == 0) slot = atomicAdd(&sh.count, total);
-        slot = __shfl_sync(0xffffffffu, slot, 0);
-        const uint32_t lt = lanemask_lt();
-        uint32_t o = slot + __popc(b0 & lt);
-        if (p0 && o < (uint32_t)cap) buf[o] = ((uint64_t)u0 << 32) | (uint32_t)c;
-        o = slot + __popc(b0) + __popc(b1 & lt);
-        if (p1 && o < (uint32_t)cap) buf[o] = ((uint64_t)u1 << 32) | (uint32_t)(c + 1);
-        o = slot + __popc(b0) + __popc(b1) + __popc(b2 & lt);
-        if (p2 && o < (uint32_t)cap) buf[o] = ((uint64_t)u2 << 32) | (uint32_t)(c + 2);
-        o = slot + __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3 & lt);
-        if (p3 && o < (uint32_t)cap) buf[o] = ((uint64_t)u3 << 32) | (uint32_t)(c + 3);
+        if (total != 0) {
+            if (lane == 0) slot = atomicAdd(&sh.count, total);
+            slot = __shfl_sync(0xffffffffu, slot, 0);
+        }
+        return slot + excl;
     };
     const float* s = src + c0;
     const int len = c1 - c0;
     const bool vec = (reinterpret_cast<uintptr_t>(s) & 15) == 0;
     const int n4 = vec ? (len >> 2) : 0;
     const float4* s4 = reinterpret_cast<const float4*>(s);
-    constexpr int U = 8;   // 16-byte loads in flight per thread
+    constexpr int U = 4;   // 16-byte loads in flight per thread
     for (int i4 = warp * 32; i4 < n4; i4 += U * NT) {   // warp-uniform trip count
         float4 x[U];
 #pragma unroll
@@ -277,16 +278,49 @@ __device__ __forceinline__ void sel_append(const float* src, int c0, int c1, uin
             const int i = i4 + u * NT + lane;
             x[u] = i < n4 ? __ldg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        uint32_t key[U][4];
+        uint32_t cnt = 0;
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int i = i4 + u * NT + lane;
-            keep4(x[u], c0 + 4 * i, i < n4 ? 4 : 0);
+            const bool ok = i4 + u * NT + lane < n4;
+            key[u][0] = ok ? score_key(x[u].x) : 0u;
+            key[u][1] = ok ? score_key(x[u].y) : 0u;
+            key[u][2] = ok ? score_key(x[u].z) : 0u;
+            key[u][3] = ok ? score_key(x[u].w) : 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) cnt += key[u][e] >= t1;
+        }
+        uint32_t total;
+        uint32_t o = warp_slots(cnt, total);
+        if (total == 0) continue;
+        const uint32_t col0 = (uint32_t)(c0 + 4 * (i4 + lane));
+        if (o + cnt <= (uint32_t)cap) {
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const bool pass = key[u][e] >= t1;
+                    if (pass) buf[o] = ((uint64_t)key[u][e] << 32) | (col0 + 4 * u * NT + e);
+                    o += pass;
+                }
+        } else {
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const bool pass = key[u][e] >= t1;
+                    if (pass && o < (uint32_t)cap) buf[o] = ((uint64_t)key[u][e] << 32) | (col0 + 4 * u * NT + e);
+                    o += pass;
+                }
         }
     }
     for (int j0 = 4 * n4 + warp * 32; j0 < len; j0 += NT) {   // tail (or the whole range if unaligned)
         const int j = j0 + lane;
-        const float v0 = j < len ? __ldg(s + j) : 0.f;
-        keep4(make_float4(v0, 0.f, 0.f, 0.f), c0 + j, j < len ? 1 : 0);
+        const uint32_t u0 = j < len ? score_key(__ldg(s + j)) : 0u;
+        const bool pass = u0 >= t1;
+        uint32_t total;
+        const uint32_t o = warp_slots(pass ? 1u : 0u, total);
+        if (pass && o < (uint32_t)cap) buf[o] = ((uint64_t)u0 << 32) | (uint32_t)(c0 + j);
     }
 }
 
@@ -428,7 +462,7 @@ __device__ __forceinline__ void sel_emit(const SelectArgs& a, const RowDesc& rd,
 
 // One CTA per row: steps 1-4 above.
 template <int NT>
-__global__ void __launch_bounds__(NT) select_stream_kernel(SelectArgs a)
+__global__ void __launch_bounds__(NT, 1024 / NT) select_stream_kernel(SelectArgs a)
 {
     extern __shared__ __align__(16) uint8_t sel_smem[];
     uint32_t* sample = reinterpret_cast<uint32_t*>(sel_smem);
@@ -472,7 +506,7 @@ __global__ void __launch_bounds__(NT) select_stream_kernel(SelectArgs a)
 // CTA of the row to finish (ticket ctr[2r + 1]) ranks the buffer and writes the row (steps
 // 3-4), then zeroes the row's two counters.  ctr must be zero at launch.
 template <int NT>
-__global__ void __launch_bounds__(NT) select_split_kernel(SelectArgs a, uint64_t* gbuf, uint32_t* ctr, int P)
+__global__ void __launch_bounds__(NT, 1024 / NT) select_split_kernel(SelectArgs a, uint64_t* gbuf, uint32_t* ctr, int P)
 {
     extern __shared__ __align__(16) uint8_t sel_smem[];
     uint32_t* sample = reinterpret_cast<uint32_t*>(sel_smem);
