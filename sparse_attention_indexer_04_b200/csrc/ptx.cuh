@@ -23,6 +23,13 @@ __device__ __forceinline__ uint64_t global_timer_ns()
     return t;
 }
 
+// Starts a bulk copy of [p, p + bytes) from global memory into L2 (a hint: nothing to wait for).
+// p 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)

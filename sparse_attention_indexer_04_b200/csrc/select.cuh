@@ -23,6 +23,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace dsa {
 
@@ -178,6 +179,18 @@ __device__ __forceinline__ uint32_t radix_select(Get get, int count, int& krem, 
     }
     block_key_range<NT>(lo, hi, scratch);
     return radix_select_in<NT>(get, count, krem, lo, hi, hist, scratch, stop_bits);
+}
+
+// Starts bringing the scores [p, p + count) into L2 while the row's first steps run (the candidate
+// scan then reads L2 instead of waiting on DRAM): 64 KB pieces, one per thread of the first few.
+// Skipped for rows not 16-byte aligned; the last partial 16 bytes are left out.
+__device__ __forceinline__ void prefetch_row_l2(const float* p, int64_t count)
+{
+    if ((reinterpret_cast<uintptr_t>(p) & 15) != 0) return;
+    const int64_t bytes = (count * 4) & ~15ll;
+    constexpr int64_t kPiece = 65536;
+    const int64_t off = (int64_t)threadIdx.x * kPiece;
+    if (off < bytes) prefetch_l2_bulk(reinterpret_cast<const char*>(p) + off, (uint32_t)min(kPiece, bytes - off));
 }
 
 // Shared scalars of one selection CTA.
@@ -481,6 +494,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_stream_kernel(SelectArgs
     const float* src = a.S + (int64_t)(a.src_from_list ? rd.list : r) * a.ld_s;
     const int nwords = (n + 31) >> 5;
     uint32_t* eqmap = gtmap + nwords;
+    if (n > k) prefetch_row_l2(src, n);
 
     for (int w = threadIdx.x; w < 2 * nwords; w += NT) gtmap[w] = 0;
     int krem = n;   // ties at T still to take (every column when n <= k)
@@ -526,9 +540,10 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_split_kernel(SelectArgs 
     uint64_t* g = gbuf + (int64_t)r * cap;
 
     if (n > k) {
-        const uint32_t tau = sel_threshold<NT>(src, n, k, cap, sample, sh);
         const int chunk = ((n + P - 1) / P + 127) & ~127;
         const int c0 = min(n, p * chunk), c1 = min(n, c0 + chunk);
+        prefetch_row_l2(src + c0, c1 - c0);
+        const uint32_t tau = sel_threshold<NT>(src, n, k, cap, sample, sh);
         if (tid == 0) sh.count = 0;
         __syncthreads();
         sel_append<NT>(src, c0, c1, tau, buf, cap, sh);
