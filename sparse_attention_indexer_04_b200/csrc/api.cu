@@ -206,20 +206,25 @@ dsa_status launch_score(const RowDesc* rows, int32_t n_rows, int32_t max_cols, c
 // candidate selection (512 best).
 int select_threads(int32_t n_rows, int32_t k) { return n_rows < 2 * 148 || k >= 4096 ? 512 : 256; }
 
+// Dynamic shared memory the select kernels may take: a CTA's 227 KB less their static shared
+// memory (SelScalars: the radix histogram and scalars, about 1.2 KB; 4 KB reserved).
+constexpr size_t kSelectDynMax = (size_t)227 * 1024 - 4096;
+static_assert(sizeof(SelScalars<512>) + 512 <= 4096, "select static shared memory");
+
 // Candidate buffer entries of the select: 1.75 k, or what fits in shared memory next to the
 // bitmaps of max_cols columns (a smaller buffer only sends more rows down the full-row path).
 int32_t select_cap(int32_t k, int32_t max_cols)
 {
-    const size_t fixed = select_smem_bytes(std::max(max_cols, 1), 0, k) + 2048;
-    const int fit = (int)(((size_t)227 * 1024 - fixed) / 8) & ~255;
+    const size_t fixed = select_smem_bytes(std::max(max_cols, 1), 0, k);
+    const int fit = fixed < kSelectDynMax ? (int)((kSelectDynMax - fixed) / 8) & ~255 : 0;
     return std::max(256, std::min(select_buf_cap(k), fit));
 }
 
 // Whether rows of max_cols columns fit the select's shared memory (sample, a candidate buffer of
-// at least 256 entries, two column bitmaps): up to about 760,000 columns.
+// at least 256 entries, two column bitmaps): up to about 770,000 columns.
 bool select_fits(int32_t k, int32_t max_cols)
 {
-    return select_smem_bytes(std::max(max_cols, 1), select_cap(k, max_cols), k) <= (size_t)227 * 1024;
+    return select_smem_bytes(std::max(max_cols, 1), select_cap(k, max_cols), k) <= kSelectDynMax;
 }
 
 // Scratch of the split-row select: two counters per row in the workspace header (zero between

@@ -80,16 +80,6 @@ __host__ __device__ inline size_t select_smem_bytes(int max_cols, int buf_cap, i
     return select_sample_bytes(max_cols, k) + (size_t)buf_cap * 8 + 2 * words * 4;
 }
 
-// Exact rank selection among `count` keys given by get(i): returns the key T
-// holding rank `krem` (1 = largest) and, in krem, how many keys equal to T
-// that rank reaches.  Digits are taken from (key - min), starting at the
-// highest bit where min and max differ, 8 bits at a time, so even the first
-// pass spreads the keys over many bins.  When the rank falls in a bin whose
-// keys are all taken, the passes stop there and the result says "every key
-// >= the bin's lower edge": T = that edge - 1 and krem = 0 (no tie at T is
-// taken).  With stop_bits > 0 only the top stop_bits bits of (key - min) are
-// resolved and the lower edge of that bin is returned: a key <= T (krem is
-// then meaningless).  All threads call it.
 // Block-wide min and max of the keys each thread passes in (lo, hi): every thread gets the result.
 // Ends with a barrier, so shared-memory writes made before the call are visible after it.
 template <int NT>
@@ -108,6 +98,17 @@ __device__ __forceinline__ void block_key_range(uint32_t& lo, uint32_t& hi, uint
     for (int w = 1; w < kSelWarps; ++w) { lo = min(lo, scratch[w]); hi = max(hi, scratch[kSelWarps + w]); }
 }
 
+// Exact rank selection among `count` keys given by get(i): returns the key T
+// holding rank `krem` (1 = largest) and, in krem, how many keys equal to T
+// that rank reaches.  Digits are taken from (key - min), starting at the
+// highest bit where min and max differ, 8 bits at a time, so even the first
+// pass spreads the keys over many bins.  When the rank falls in a bin whose
+// keys are all taken, the passes stop there and the result says "every key
+// >= the bin's lower edge": T = that edge - 1 and krem = 0 (no tie at T is
+// taken).  With stop_bits > 0 only the top stop_bits bits of (key - min) are
+// resolved and the lower edge of that bin is returned: a key <= T (krem is
+// then meaningless).  All threads call it.
+//
 // radix_select with the keys' block-wide range [lo, hi] already known (all threads pass the same).
 template <int NT, typename Get>
 __device__ __forceinline__ uint32_t radix_select_in(Get get, int count, int& krem, uint32_t lo, uint32_t hi,

@@ -43,3 +43,12 @@ def test_largest_hisa_block_and_keep():
     ref = oracle.hisa(b, 256, 256, 64)
     check_exact_sets(kept, ref["kept"], "kept")
     check_exact_sets(idx, ref["idx"], "idx")
+
+
+def test_longest_supported_row():
+    """Rows of 757,000 keys, just under the longest the selection's shared memory holds (two column
+    bitmaps next to the sample and a candidate buffer clamped to 256 entries): exact all the same."""
+    b = workloads.ragged(74, [2], [757000], H=4, d=32, k=64, integer=True)
+    idx = Dev(b).topk(64)
+    ascending_packed(idx)
+    check_exact_sets(idx, oracle.dense(b, k=64)["idx"])
