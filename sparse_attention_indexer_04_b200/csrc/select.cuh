@@ -248,19 +248,22 @@ __device__ __forceinline__ uint32_t sel_threshold(const float* src, int n, int k
     return radix_select_in<NT>([&](int i) { return sample[i]; }, m, rank, lo, hi, sh.hist, sh.scratch, 16);
 }
 
-// 2. Appends (key << 32 | column) of every column c in [c0, c1) whose key is >= max(tau, 1) to
-// buf; sh.count (zero on entry) counts them all, entries past cap are dropped.  (Key 0 is a NaN
-// with every bit set; leaving it out keeps the buffer exact: with k entries or more, the k-th
-// largest is >= 1.)  c0 is a multiple of 4.  Each thread loads 16 columns per round; a warp
-// finds its threads' output offsets by one prefix count over the threads' pass counts (five
-// ballots on the count's bits), takes one shared atomic, and each thread writes its passing
-// columns at consecutive slots.
+// 2. Appends (score bits << 32 | column) of every column c in [c0, c1) whose key is >= max(tau, 1)
+// to buf; sh.count (zero on entry) counts them all, entries past cap are dropped.  (Key 0 is a
+// NaN with every bit set; leaving it out keeps the buffer exact: with k entries or more, the
+// k-th largest is >= 1.)  The test is made on the float itself against the float whose key is
+// max(tau, 1) (-inf when that key is at or below -inf's): for every non-NaN score the two agree,
+// -0 and +0 included.  sel_buf_keys turns the stored scores into keys.  c0 is a multiple of 4.
+// Each thread loads 16 columns per round; a warp finds its threads' output offsets by one prefix
+// count over the threads' pass counts (five ballots on the count's bits), takes one shared
+// atomic, and each thread writes its passing columns at consecutive slots.
 template <int NT>
 __device__ __forceinline__ void sel_append(const float* src, int c0, int c1, uint32_t tau, uint64_t* buf, int cap,
                                            SelScalars<NT>& sh)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t t1 = max(tau, 1u);
+    const float tf = t1 <= 0x007fffffu ? -INFINITY : key_score(t1);   // 0x007fffff: the key of -inf
     const uint32_t lt = lanemask_lt();
     // A warp's slots for `cnt` entries of this lane (cnt < 32), in lane order; returns the first.
     auto warp_slots = [&](uint32_t cnt, uint32_t& total) {
@@ -292,17 +295,17 @@ __device__ __forceinline__ void sel_append(const float* src, int c0, int c1, uin
             const int i = i4 + u * NT + lane;
             x[u] = i < n4 ? __ldg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        uint32_t key[U][4];
+        float v[U][4];
         uint32_t cnt = 0;
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const bool ok = i4 + u * NT + lane < n4;
-            key[u][0] = ok ? score_key(x[u].x) : 0u;
-            key[u][1] = ok ? score_key(x[u].y) : 0u;
-            key[u][2] = ok ? score_key(x[u].z) : 0u;
-            key[u][3] = ok ? score_key(x[u].w) : 0u;
+            v[u][0] = x[u].x; v[u][1] = x[u].y; v[u][2] = x[u].z; v[u][3] = x[u].w;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) cnt += key[u][e] >= t1;
+            for (int e = 0; e < 4; ++e) {
+                if (!ok) v[u][e] = __int_as_float(0x7fffffff);   // NaN: never passes
+                cnt += v[u][e] >= tf;
+            }
         }
         uint32_t total;
         uint32_t o = warp_slots(cnt, total);
@@ -313,8 +316,8 @@ __device__ __forceinline__ void sel_append(const float* src, int c0, int c1, uin
             for (int u = 0; u < U; ++u)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const bool pass = key[u][e] >= t1;
-                    if (pass) buf[o] = ((uint64_t)key[u][e] << 32) | (col0 + 4 * u * NT + e);
+                    const bool pass = v[u][e] >= tf;
+                    if (pass) buf[o] = ((uint64_t)__float_as_uint(v[u][e]) << 32) | (col0 + 4 * u * NT + e);
                     o += pass;
                 }
         } else {
@@ -322,35 +325,56 @@ __device__ __forceinline__ void sel_append(const float* src, int c0, int c1, uin
             for (int u = 0; u < U; ++u)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const bool pass = key[u][e] >= t1;
-                    if (pass && o < (uint32_t)cap) buf[o] = ((uint64_t)key[u][e] << 32) | (col0 + 4 * u * NT + e);
+                    const bool pass = v[u][e] >= tf;
+                    if (pass && o < (uint32_t)cap)
+                        buf[o] = ((uint64_t)__float_as_uint(v[u][e]) << 32) | (col0 + 4 * u * NT + e);
                     o += pass;
                 }
         }
     }
     for (int j0 = 4 * n4 + warp * 32; j0 < len; j0 += NT) {   // tail (or the whole range if unaligned)
         const int j = j0 + lane;
-        const uint32_t u0 = j < len ? score_key(__ldg(s + j)) : 0u;
-        const bool pass = u0 >= t1;
+        const float v0 = j < len ? __ldg(s + j) : __int_as_float(0x7fffffff);
+        const bool pass = v0 >= tf;
         uint32_t total;
         const uint32_t o = warp_slots(pass ? 1u : 0u, total);
-        if (pass && o < (uint32_t)cap) buf[o] = ((uint64_t)u0 << 32) | (uint32_t)(c0 + j);
+        if (pass && o < (uint32_t)cap) buf[o] = ((uint64_t)__float_as_uint(v0) << 32) | (uint32_t)(c0 + j);
     }
 }
 
-// 3. Marks the row's top k in the bitmaps (> T in gtmap, == T in eqmap, both zeroed) and returns
-// in krem how many ties at T to take.  From the candidate buffer when it holds every column
-// with key >= tau (k <= count <= cap), else (a misleading sample) by radix passes over the
-// whole row.
+// Turns the buffer's first count entries from (score bits, column) into (key, column) and returns
+// the keys' block-wide range (every thread; ends with a barrier).
 template <int NT>
-__device__ __forceinline__ void sel_mark(const float* src, int n, int k, const uint64_t* buf, int count, int cap,
+__device__ __forceinline__ void sel_buf_keys(uint64_t* buf, int count, uint32_t& lo, uint32_t& hi,
+                                             SelScalars<NT>& sh)
+{
+    lo = 0xffffffffu;
+    hi = 0u;
+    for (int i = threadIdx.x; i < count; i += NT) {
+        const uint64_t e = buf[i];
+        const uint32_t u = score_key(__uint_as_float((uint32_t)(e >> 32)));
+        buf[i] = ((uint64_t)u << 32) | (uint32_t)e;
+        lo = min(lo, u);
+        hi = max(hi, u);
+    }
+    block_key_range<NT>(lo, hi, sh.scratch);
+}
+
+// 3. Marks the row's top k in the bitmaps (> T in gtmap, == T in eqmap, both zeroed) and returns
+// in krem how many ties at T to take.  From the candidate buffer (score bits, turned into keys
+// here) when it holds every column with key >= tau (k <= count <= cap), else (a misleading
+// sample) by radix passes over the whole row.
+template <int NT>
+__device__ __forceinline__ void sel_mark(const float* src, int n, int k, uint64_t* buf, int count, int cap,
                                          int& krem, uint32_t* gtmap, uint32_t* eqmap, SelScalars<NT>& sh)
 {
     const int tid = threadIdx.x;
     krem = k;
     if (count >= k && count <= cap) {
-        const uint32_t thresh =
-            radix_select<NT>([&](int i) { return (uint32_t)(buf[i] >> 32); }, count, krem, sh.hist, sh.scratch);
+        uint32_t lo, hi;
+        sel_buf_keys<NT>(buf, count, lo, hi, sh);
+        const uint32_t thresh = radix_select_in<NT>([&](int i) { return (uint32_t)(buf[i] >> 32); }, count, krem,
+                                                    lo, hi, sh.hist, sh.scratch);
         for (int i = tid; i < count; i += NT) {
             const uint32_t u = (uint32_t)(buf[i] >> 32), c = (uint32_t)buf[i];
             if (u > thresh) atomicOr(&gtmap[c >> 5], 1u << (c & 31));
