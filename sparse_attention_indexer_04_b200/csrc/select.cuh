@@ -437,6 +437,10 @@ __device__ __forceinline__ void sel_emit(const SelectArgs& a, const RowDesc& rd,
     const uint32_t g_before = (uint32_t)(before >> 32), e_before = (uint32_t)before;
     uint32_t out = g_before + min(e_before, (uint32_t)krem);   // ties before this thread are taken first
     int left_e = (int)min(ne, (uint32_t)max(0, krem - (int)e_before));
+    // the key of column w * 32 + b is wbase + b (identity map, and block maps whose blocks are whole
+    // bitmap words), else list[w * 32 + b] (list maps) or map_col (other block sizes)
+    const int32_t* lrow = a.map.kind == kMapIdentity ? nullptr : a.map.list + (int64_t)rd.list * a.map.list_ld;
+    const bool per_word = a.map.kind == kMapIdentity || (a.map.kind == kMapBlocks && (a.map.block & 31) == 0);
     for (int w = w0; w < w1; ++w) {
         uint32_t e = eqmap[w], te = 0;
         for (; left_e > 0 && e; --left_e) {   // the lowest remaining ties
@@ -444,9 +448,16 @@ __device__ __forceinline__ void sel_emit(const SelectArgs& a, const RowDesc& rd,
             te |= low;
             e ^= low;
         }
-        for (uint32_t bits = gtmap[w] | te; bits; bits &= bits - 1) {
-            const int col = w * 32 + __ffs(bits) - 1;
-            const int32_t key = map_col(a.map, rd, col);
+        uint32_t bits = gtmap[w] | te;
+        if (!bits) continue;
+        const int c0 = w * 32;
+        const int32_t wbase = a.map.kind == kMapIdentity ? c0 + a.map.offset
+                              : per_word ? lrow[c0 / a.map.block] * a.map.block + c0 % a.map.block
+                                         : 0;
+        for (; bits; bits &= bits - 1) {
+            const int b = __ffs(bits) - 1;
+            const int col = c0 + b;
+            const int32_t key = per_word ? wbase + b : a.map.kind == kMapList ? lrow[col] : map_col(a.map, rd, col);
             const float sc = osc ? key_score(score_key(__ldg(src + col))) : 0.f;
             if (staged) {
                 stage[out] = key;
