@@ -38,7 +38,7 @@
  *  Supported shapes.  H a power of two in 1..64; d in {32, 64, 128};
  *  1 <= k <= 16384; a ranked row (a sequence's keys for the dense top-k and
  *  PIVOT's proxy scan, its middle blocks for HISA's block filter) of at most
- *  about 770,000 columns: the selection keeps two bitmaps of the row's
+ *  774,144 columns (for k below 16,128; a little more above): the selection keeps two bitmaps of the row's
  *  columns in shared memory.  Otherwise DSA_ERR_UNSUPPORTED.
  *  Ownership.  The caller owns every buffer: inputs, outputs and the
  *  workspace.  The library allocates no device memory, never synchronises

@@ -221,7 +221,7 @@ int32_t select_cap(int32_t k, int32_t max_cols)
 }
 
 // Whether rows of max_cols columns fit the select's shared memory (sample, a candidate buffer of
-// at least 256 entries, two column bitmaps): up to about 770,000 columns.
+// at least 256 entries, two column bitmaps): up to 774,144 columns.
 bool select_fits(int32_t k, int32_t max_cols)
 {
     return select_smem_bytes(std::max(max_cols, 1), select_cap(k, max_cols), k) <= kSelectDynMax;

@@ -100,6 +100,15 @@ def test_argument_errors_return_before_any_launch():
     assert call_topk(host_layout([1], [1_000_000]), k=2048) == 2
 
 
+def test_longest_row_boundary():
+    """The selection's shared memory (227 KB less 4 KB for its static part) holds the 8192-entry
+    sample, a 256-entry candidate buffer and two bitmaps of ceil(n / 32) words: 774,144 columns fit,
+    one more does not.  The shape check comes before the workspace check, so a row that fits
+    reaches the workspace error (3) and one that does not is refused as unsupported (2)."""
+    assert call_topk(host_layout([1], [774_144]), k=2048, ws_bytes=16) == 3
+    assert call_topk(host_layout([1], [774_145]), k=2048, ws_bytes=16) == 2
+
+
 def test_host_entry_argument_errors_need_no_gpu():
     lib = dsa.library()
     lay = host_layout([8], [8])
