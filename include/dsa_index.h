@@ -38,8 +38,9 @@
  *  Supported shapes.  H a power of two in 1..64; d in {32, 64, 128};
  *  1 <= k <= 16384; a ranked row (a sequence's keys for the dense top-k and
  *  PIVOT's proxy scan, its middle blocks for HISA's block filter) of at most
- *  774,144 columns (for k below 16,128; a little more above): the selection keeps two bitmaps of the row's
- *  columns in shared memory.  Otherwise DSA_ERR_UNSUPPORTED.
+ *  774,144 columns (for k below 16,128; a little more above): the selection
+ *  keeps two bitmaps of the row's columns in shared memory.  Otherwise
+ *  DSA_ERR_UNSUPPORTED.
  *  Ownership.  The caller owns every buffer: inputs, outputs and the
  *  workspace.  The library allocates no device memory, never synchronises
  *  the stream (dsa_device_check and dsa_profile_read excepted) and keeps no
