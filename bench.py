@@ -245,10 +245,38 @@ class Hisa:
                             idx=self.idx, ws=self.ws)
 
 
+def graph_times(step, steps, flush):
+    """The step captured once in a CUDA graph: mean device time (us) of a replay with L2 flushed before
+    it, and of back-to-back replays (each launch's host latency hidden, as a serving loop would)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            step()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        g.replay()
+    flushed = time_steps(g.replay, steps, flush)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = 4 * steps
+    e0.record()
+    for _ in range(n):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    out = {"us_per_step_l2_flushed": round(1e3 * sum(flushed) / steps, 2),
+           "us_per_step_back_to_back": round(1e3 * e0.elapsed_time(e1) / n, 2)}
+    del g
+    return out
+
+
 def secondary(device, flush, steps, only=None, pivot_T=131072):
     out = {}
 
-    def run(name, make, extra):
+    def run(name, make, extra, graph=False):
         if only and only not in name:
             return
         try:
@@ -259,6 +287,11 @@ def secondary(device, flush, steps, only=None, pivot_T=131072):
             ms = time_steps(step, steps, flush)
             r = {"us_per_step": round(1e3 * sum(ms) / steps, 2), "steps": steps, "setup_s": round(time.time() - t0, 1)}
             r.update(extra(step, sum(ms) / steps))
+            if graph:
+                try:
+                    r["cuda_graph"] = graph_times(step, steps, flush)
+                except Exception as e:  # the eager numbers stand without it
+                    r["cuda_graph"] = {"error": f"{type(e).__name__}: {e}"[:200]}
             step.dsa.profile_enable(True)                      # a second, separately timed pass per kernel
             time_steps(step, steps, flush)
             prof = step.dsa.profile_read()
@@ -277,9 +310,10 @@ def secondary(device, flush, steps, only=None, pivot_T=131072):
         gbs = step.alg_bytes() / (ms * 1e-3) / 1e9
         return {"alg_bytes": step.alg_bytes(), "achieved_gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
 
-    run("dense_decode_B16_L32768_mtp2", lambda: DenseTopk(workloads.dense_decode(seed=1), device), dec_extra)
+    run("dense_decode_B16_L32768_mtp2", lambda: DenseTopk(workloads.dense_decode(seed=1), device), dec_extra,
+        graph=True)
     run("dense_decode_B16_L131072_mtp2", lambda: DenseTopk(workloads.dense_decode(seed=1, L=131072), device),
-        dec_extra)
+        dec_extra, graph=True)
     if not only or "pivot" in only or "reuse" in only or "refine" in only:
         pv = workloads.pivot_prefill(seed=3, T=pivot_T)
         dense_pairs = pv.eligible_pairs()
@@ -287,7 +321,8 @@ def secondary(device, flush, steps, only=None, pivot_T=131072):
             run(f"pivot_prefill_T{pivot_T}_G16_C8192_{name}", lambda m=mode: Pivot(pv, device, m),
                 lambda step, ms: {"dense_equiv_gpairs_s": round(dense_pairs / (ms * 1e-3) / 1e9, 2)})
         del pv
-    run("hisa_decode_B4_L262144_keep64", lambda: Hisa(workloads.hisa_decode(seed=4), device), lambda s, ms: {})
+    run("hisa_decode_B4_L262144_keep64", lambda: Hisa(workloads.hisa_decode(seed=4), device), lambda s, ms: {},
+        graph=True)
     return out
 
 
