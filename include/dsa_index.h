@@ -132,15 +132,17 @@ dsa_status dsa_index_topk(const dsa_batch* batch, const void* Q, const void* K, 
  * Q, K, W, q_pos_host and idx are HOST pointers (page-locked for the copies
  * to overlap; pageable memory works but serialises); batch->q_offsets_host
  * and k_offsets_host are used and the batch's device pointer fields are
- * ignored.  The rows are processed in the same chunks as dsa_index_topk:
- * while chunk c is scored and selected on `stream`, chunk c+1's queries are
- * copied in on `in_stream` and chunk c-1's indices copied out on
+ * ignored.  The rows are cut into chunks (about eight, of at least 2048
+ * rows, within dsa_index_topk's score buffer) taken in order of decreasing
+ * work (eligible pairs, counted on the host from q_pos_host): while one
+ * chunk is scored and selected on `stream`, the next two chunks' queries are
+ * copied in on `in_stream` and earlier chunks' indices copied out on
  * `out_stream` (K, W and q_pos are copied once, first).  in_stream and
  * out_stream must differ from `stream` (they may be the same stream, which
  * serialises the two directions).  Returns after enqueueing; idx is
  * complete when `stream` has passed the call's work.  The workspace
  * (dsa_index_topk_host_workspace bytes) holds dsa_index_topk's workspace
- * followed by device copies of K, W, q_pos, the offsets and two chunks of
+ * followed by device copies of K, W, q_pos, the offsets and three chunks of
  * queries and of indices.  The status word is at the workspace start as
  * for every call.
  */

@@ -551,18 +551,31 @@ size_t dense_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k,
 }
 
 // Workspace of dsa_index_topk_host: dsa_index_topk's workspace first (its header stays at the
-// base), then device copies of the inputs and two row chunks' queries and indices.
+// base), then device copies of the inputs and kHostBufs row chunks' queries and indices.
+constexpr int kHostBufs = 3;
+constexpr int32_t kHostChunks = 8;        // row chunks a large batch is cut into
+constexpr int32_t kHostMinChunk = 2048;   // rows per chunk at least
+
 struct HostPlan {
     int32_t* q_off;
     int32_t* k_off;
     int32_t* q_pos;
     uint8_t* K;
     float* W;
-    uint8_t* Q[2];
-    int32_t* idx[2];
+    uint8_t* Q[kHostBufs];
+    int32_t* idx[kHostBufs];
     RowDesc* rows;   // one chunk's rows, query rows relative to the chunk
     int32_t chunk;
 };
+
+// Rows per chunk of the host-memory entry point: about kHostChunks chunks of at least kHostMinChunk
+// rows (the copies of one chunk then overlap the work of another), and no more than the score
+// buffer holds.
+int32_t host_chunk_rows(int32_t nq, int64_t ld)
+{
+    const int32_t want = std::max(kHostMinChunk, (nq + kHostChunks - 1) / kHostChunks);
+    return std::max(1, std::min(chunk_rows(nq, ld), want));
+}
 
 size_t host_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, DensePlan* dp, HostPlan* p)
 {
@@ -571,13 +584,13 @@ size_t host_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, 
     c.off = align256(inner);
     const int32_t nq = std::max(1, b->num_queries);
     const size_t qrow_bytes = size_t(b->num_heads) * b->head_dim * 2;
-    p->chunk = chunk_rows(nq, score_ld(hi.max_k));
+    p->chunk = host_chunk_rows(nq, score_ld(hi.max_k));
     p->q_off = c.take<int32_t>(b->num_seqs + 1);
     p->k_off = c.take<int32_t>(b->num_seqs + 1);
     p->q_pos = c.take<int32_t>(nq);
     p->K = c.take<uint8_t>(size_t(std::max(1, b->num_keys)) * b->head_dim * 2);
     p->W = c.take<float>(size_t(nq) * b->num_heads);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kHostBufs; ++i) {
         p->Q[i] = c.take<uint8_t>(size_t(p->chunk) * qrow_bytes);
         p->idx[i] = c.take<int32_t>(size_t(p->chunk) * k);
     }
@@ -879,8 +892,23 @@ dsa_status dsa_index_topk_host(const dsa_batch* b, const int32_t* q_pos_host, co
     const int H = b->num_heads, D = b->head_dim;
     const size_t qrow_bytes = size_t(H) * D * 2;
 
+    // Row chunks in order of decreasing work (eligible pairs, from the host-side positions): the
+    // largest are scored while the later chunks' queries still come in, and the last chunk, whose
+    // work and index copy nothing overlaps, is the smallest (for a causal prefill, the first rows).
+    const int32_t n_chunks = (nq + hp.chunk - 1) / hp.chunk;
+    auto rows_of = [&](int32_t c) { return std::min(hp.chunk, nq - c * hp.chunk); };
+    std::vector<int64_t> work(n_chunks, 0);
+    for (int32_t q = 0; q < b->num_seqs; ++q) {
+        const int32_t L = b->k_offsets_host[q + 1] - b->k_offsets_host[q];
+        for (int32_t t = b->q_offsets_host[q]; t < b->q_offsets_host[q + 1]; ++t)
+            work[t / hp.chunk] += std::min<int64_t>(L, std::max<int64_t>(0, int64_t(q_pos_host[t]) + 1));
+    }
+    std::vector<int32_t> order(n_chunks);
+    for (int32_t c = 0; c < n_chunks; ++c) order[c] = c;
+    std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t c) { return work[a] > work[c]; });
+
     // Events linking the streams (released once the device has passed them).
-    constexpr int kEvents = 9;
+    constexpr int kEvents = 3 + 3 * kHostBufs;
     cudaEvent_t ev[kEvents];
     int made = 0;
     for (; made < kEvents; ++made)
@@ -888,20 +916,22 @@ dsa_status dsa_index_topk_host(const dsa_batch* b, const int32_t* q_pos_host, co
     auto release = [&]() { for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]); };
     if (made < kEvents) { release(); return DSA_ERR_CUDA; }
     cudaEvent_t e_start = ev[0], e_in = ev[1], e_out = ev[2];
-    cudaEvent_t e_q[2] = {ev[3], ev[4]}, e_done[2] = {ev[5], ev[6]}, e_back[2] = {ev[7], ev[8]};
+    cudaEvent_t* e_q = ev + 3;                   // chunk's queries arrived in its buffer
+    cudaEvent_t* e_done = ev + 3 + kHostBufs;    // chunk scored and selected: its query buffer is free
+    cudaEvent_t* e_back = ev + 3 + 2 * kHostBufs;   // chunk's indices copied out: its index buffer is free
     bool ok = true;
     auto chk = [&](cudaError_t e) { ok = ok && e == cudaSuccess; };
-    const int32_t n_chunks = (nq + hp.chunk - 1) / hp.chunk;
-    auto rows_of = [&](int32_t c) { return std::min(hp.chunk, nq - c * hp.chunk); };
-    // query rows of chunk c into buffer c % 2, once chunk c - 2 no longer reads it
-    auto send_queries = [&](int32_t c) {
-        if (c >= 2) chk(cudaStreamWaitEvent(si, e_done[c & 1], 0));
-        chk(cudaMemcpyAsync(hp.Q[c & 1], static_cast<const uint8_t*>(Q) + size_t(c) * hp.chunk * qrow_bytes,
+    // the queries of the p-th chunk in processing order into buffer p % kHostBufs, once the chunk
+    // kHostBufs earlier no longer reads it
+    auto send_queries = [&](int32_t p) {
+        const int32_t c = order[p], x = p % kHostBufs;
+        if (p >= kHostBufs) chk(cudaStreamWaitEvent(si, e_done[x], 0));
+        chk(cudaMemcpyAsync(hp.Q[x], static_cast<const uint8_t*>(Q) + size_t(c) * hp.chunk * qrow_bytes,
                             size_t(rows_of(c)) * qrow_bytes, cudaMemcpyHostToDevice, si));
-        chk(cudaEventRecord(e_q[c & 1], si));
+        chk(cudaEventRecord(e_q[x], si));
     };
 
-    // The small inputs and the keys first (after the header is cleared), then chunk 0's queries.
+    // The small inputs and the keys first (after the header is cleared), then the first chunks' queries.
     chk(cudaEventRecord(e_start, st));
     chk(cudaStreamWaitEvent(si, e_start, 0));
     chk(cudaStreamWaitEvent(so, e_start, 0));
@@ -911,21 +941,22 @@ dsa_status dsa_index_topk_host(const dsa_batch* b, const int32_t* q_pos_host, co
     chk(cudaMemcpyAsync(hp.W, W, size_t(nq) * H * sizeof(float), cudaMemcpyHostToDevice, si));
     if (b->num_keys > 0) chk(cudaMemcpyAsync(hp.K, K, size_t(b->num_keys) * D * 2, cudaMemcpyHostToDevice, si));
     chk(cudaEventRecord(e_in, si));
-    send_queries(0);
+    for (int32_t p = 0; p < std::min<int32_t>(kHostBufs - 1, n_chunks); ++p) send_queries(p);
     chk(cudaStreamWaitEvent(st, e_in, 0));
     if (!ok) { release(); return DSA_ERR_CUDA; }
     DSA_LAUNCH(kProfSetup, st, dense_rows_kernel<<<(nq + 255) / 256, 256, 0, st>>>(d.q_offsets, d.k_offsets, d.q_pos,
                                                                                   d.num_seqs, nq, dp.rows));
     if ((s = launched()) != DSA_OK) { release(); return s; }
 
-    // Row chunks: while chunk c is scored and selected, chunk c+1's queries come in and chunk c-1's
-    // indices go out.
+    // While one chunk is scored and selected, the next chunks' queries come in and the previous
+    // chunks' indices go out.
     const int64_t ld = score_ld(hi.max_k);
-    for (int32_t c = 0; c < n_chunks && ok; ++c) {
-        const int32_t r0 = c * hp.chunk, nr = rows_of(c);
-        const int x = c & 1;
+    for (int32_t p = 0; p < n_chunks && ok; ++p) {
+        const int32_t c = order[p], r0 = c * hp.chunk, nr = rows_of(c);
+        const int x = p % kHostBufs;
+        if (p + kHostBufs - 1 < n_chunks) send_queries(p + kHostBufs - 1);
         chk(cudaStreamWaitEvent(st, e_q[x], 0));
-        if (c >= 2) chk(cudaStreamWaitEvent(st, e_back[x], 0));   // chunk c-2's indices have left idx[x]
+        if (p >= kHostBufs) chk(cudaStreamWaitEvent(st, e_back[x], 0));   // its index buffer has been copied out
         DSA_LAUNCH(kProfSetup, st, chunk_rows_kernel<<<(nr + 255) / 256, 256, 0, st>>>(dp.rows, r0, nr, hp.rows));
         if ((s = launched()) != DSA_OK) break;
         const TcSource src{hp.Q[x], nr, hp.W + size_t(r0) * H, d.q_offsets, b->q_offsets_host, b->num_seqs};
@@ -935,7 +966,6 @@ dsa_status dsa_index_topk_host(const dsa_batch* b, const int32_t* q_pos_host, co
         s = launch_select(hp.rows, nr, hi.max_k, k, ColMap{}, dp.S, ld, false, hp.idx[x], k, nullptr, 0, st, dp.split);
         if (s != DSA_OK) break;
         chk(cudaEventRecord(e_done[x], st));
-        if (c + 1 < n_chunks) send_queries(c + 1);
         chk(cudaStreamWaitEvent(so, e_done[x], 0));
         chk(cudaMemcpyAsync(idx + size_t(r0) * k, hp.idx[x], size_t(nr) * k * sizeof(int32_t), cudaMemcpyDeviceToHost,
                             so));

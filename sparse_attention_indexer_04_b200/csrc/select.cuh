@@ -4,19 +4,23 @@
 // largest key of the row) plus the lowest columns whose key equals T: ties
 // go to the lower key index.  Columns are written in ascending order.
 //
-// A row is ranked in four steps:
+// A row is ranked in four steps (the CTA first starts a bulk L2 prefetch of
+// its row, so that step 2 reads L2):
 //   1. threshold: the keys of m columns (m >= 128 n / k, 2048 to 8192), in
 //      m/32 evenly spaced runs of 32, are ranked and the one at rank k*m/n
 //      plus a 4-sigma margin becomes tau (rows that fit the candidate buffer
 //      skip this and keep every column);
-//   2. one streaming pass appends every column with key >= tau to a
-//      candidate buffer (about 1.75 k entries);
+//   2. one streaming pass appends every column with key >= tau (tested on
+//      the float itself) to a candidate buffer of about 1.75 k entries, as
+//      (score bits, column);
 //   3. if at least k columns passed and none was dropped, the top k of the
-//      row are exactly the top k of the buffer: an 8-bit radix select over
-//      the buffer finds T and the number of T-ties to take.  Otherwise
-//      (a misleading sample) T is found by radix passes over the whole row;
+//      row are exactly the top k of the buffer: its scores become keys and
+//      an 8-bit radix select over it finds T and the number of T-ties to
+//      take.  Otherwise (a misleading sample) T is found by radix passes
+//      over the whole row;
 //   4. the selected columns are marked in two bitmaps (> T, == T) and emitted
-//      in column order, taking the first ties.
+//      in column order, taking the first ties; the output row is assembled in
+//      shared memory and written with 16-byte stores.
 // select_stream_kernel gives each row one CTA (many rows: prefill).
 // select_split_kernel gives each row several CTAs that share step 2 through
 // a global buffer, the last of them finishing the row (few long rows: decode).
