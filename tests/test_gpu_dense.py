@@ -165,8 +165,11 @@ def test_few_long_rows_exact(seed, q_lens, k_lens, k, mode):
 
 
 @pytest.mark.parametrize("make", [
-    lambda: workloads.dense_prefill(seed=2),                                     # 4 row chunks, pipelined
+    lambda: workloads.dense_prefill(seed=2),                                     # 8 row chunks, largest work first
     lambda: workloads.ragged(60, [5, 0, 64], [300, 17, 129], H=4, d=32, k=24),   # one chunk, ragged
+    # 5 chunks of 2048 rows over three sequences with random positions: the work order is a
+    # permutation of the row order and the three buffers rotate
+    lambda: workloads.ragged(62, [3000, 2500, 4000], [3000, 6000, 4000], H=4, d=32, k=64, pos_mode="random"),
     lambda: workloads.dense_decode(seed=61, B=4, L=5000, n_mtp=2, H=64, d=128, k=256),
 ])
 def test_host_memory_entry_matches_device_entry(make):
