@@ -14,6 +14,7 @@
 #include "score_simt.cuh"
 #include "score_tc.cuh"
 #include "select.cuh"
+#include "select_cluster.cuh"
 #include "reuse.cuh"
 #include "setup.cuh"
 
@@ -115,6 +116,29 @@ void launch_pdl(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
+    (void)cudaLaunchKernelEx(&cfg, kern, args...);   // errors surface through launched()
+}
+
+// Launches a kernel as clusters of `cluster` CTAs along x (with programmatic stream
+// serialization, as launch_pdl).
+template <typename... KArgs, typename... Args>
+void launch_clustered(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, int cluster, cudaStream_t st,
+                      Args... args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
     (void)cudaLaunchKernelEx(&cfg, kern, args...);   // errors surface through launched()
 }
 
@@ -275,6 +299,15 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
     dsa_status s;
     const int P = select_parts(n_rows, max_cols);
     if (sp.buf && sp.ctr && n_rows <= sp.max_rows && P > 1 && !n_rows_dev) {
+        // a row's CTAs as one cluster when they fit one (P <= 8) and its shared memory layout fits
+        const int chunk_words = ((((max_cols + P - 1) / P + 127) & ~127) + 31) / 32;
+        const size_t csmem = cluster_smem_bytes(a.sample_bytes, a.buf_cap, chunk_words);
+        if (P <= kClusterMaxParts && csmem <= kSelectDynMax) {
+            if ((s = set_smem(select_cluster_kernel<512>, csmem)) != DSA_OK) return s;
+            DSA_LAUNCH(kProfSelect, st, launch_clustered(select_cluster_kernel<512>, n_rows * P, 512, csmem, P, st, a,
+                                                         P, chunk_words));
+            return launched();
+        }
         if ((s = set_smem(select_split_kernel<512>, smem)) != DSA_OK) return s;
         DSA_LAUNCH(kProfSelect, st, launch_pdl(true, select_split_kernel<512>, n_rows * P, 512, smem, st, a, sp.buf,
                                                sp.ctr, P));

@@ -1,0 +1,361 @@
+// Exact per-row top-k for few long rows (decode): the P CTAs of a row form one thread-block
+// cluster (2 <= P <= 8) and share the steps of select.cuh through distributed shared memory,
+// instead of handing candidates to one finishing CTA through L2.
+//
+//   1. threshold: the row's sample (the same m/32 runs of 32 columns select_stream_kernel reads)
+//      is split among the P CTAs by runs; each counts its part into its own histogram and the
+//      leader (cluster rank 0) sums the P histograms digit by digit, so tau is the key one CTA
+//      would find over the whole sample;
+//   2. each CTA appends the columns of its chunk with key >= tau to its own candidate buffer;
+//   3. the CTAs copy their candidates into the leader's buffer (offsets from one atomic on the
+//      leader's counter); if the union holds >= k entries and nothing overflowed, the leader
+//      ranks it (T and the number of T-ties to take), otherwise it ranks the whole row itself;
+//   4. each CTA marks its own chunk (> T, == T) in its own bitmaps; the per-CTA counts go through
+//      the leader; each CTA writes its chunk's columns at its offset, the T-ties taken in column
+//      order across the chunks.
+// Every cluster barrier is reached by every thread of every CTA, in the same order: the
+// branches between barriers depend only on the row, which the whole cluster shares.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "select.cuh"
+
+namespace dsa {
+
+namespace cg = cooperative_groups;
+
+constexpr int kClusterMaxParts = 8;
+
+// Scalars the row's CTAs exchange; the leader's copy is the one read.
+struct alignas(16) ClusterShared {
+    uint32_t lo[kClusterMaxParts];   // each CTA's sample key range
+    uint32_t hi[kClusterMaxParts];
+    uint32_t gt[kClusterMaxParts];   // each CTA's marked counts (> T, == T)
+    uint32_t eq[kClusterMaxParts];
+    uint32_t step[3];                // the current radix digit: digit, keys above it, whole-digit flag
+    uint32_t count;                  // candidates in the leader's buffer
+    uint32_t overflow;               // nonzero: some buffer overflowed
+    uint32_t T;                      // the row's k-th key
+    int32_t krem;                    // ties at T to take
+    uint32_t mode;                   // 0: T from the candidates, 1: from the whole row, 2: every column
+};
+
+// Dynamic shared memory of select_cluster_kernel: the sample, the CTA's candidate buffer, the
+// leader's union buffer (cap entries each) and two bitmaps of one chunk (chunk_words words each).
+__host__ __device__ inline size_t cluster_smem_bytes(size_t sample_bytes, int cap, int chunk_words)
+{
+    return sample_bytes + (size_t)cap * 16 + (size_t)chunk_words * 8;
+}
+
+// radix_select over keys spread over the cluster's CTAs (count of them in this CTA, given by
+// get): each pass counts into the CTA's own histogram, the leader's warp 0 sums the P
+// histograms and picks the digit.  lo, hi and krem are the same in every CTA.  Two cluster
+// barriers per pass.
+template <int NT, typename Get>
+__device__ __forceinline__ uint32_t cluster_radix(cg::cluster_group& cl, ClusterShared* lead, int P, Get get,
+                                                  int count, int& krem, uint32_t lo, uint32_t hi, int stop_bits,
+                                                  SelScalars<NT>& sh)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int top = 32 - __clz(hi - lo);
+    const int stop = stop_bits > 0 ? max(top - stop_bits, 0) : 0;
+    uint32_t prefix = 0;
+    while (top > stop) {
+        const int shift = max(top - 8, 0), width = top - shift;
+        __syncthreads();
+        for (int i = tid; i < 256; i += NT) sh.hist[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < count; i += NT) {
+            const uint32_t rel = get(i) - lo;
+            if (((rel >> 1) >> (top - 1)) == prefix) atomicAdd(&sh.hist[(rel >> shift) & ((1u << width) - 1u)], 1u);
+        }
+        cl.sync();   // every CTA's histogram is complete
+        if (cl.block_rank() == 0 && warp == 0) {
+            uint32_t c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            for (int q = 0; q < P; ++q) {
+                const uint32_t* hq = cl.map_shared_rank(sh.hist, q);
+#pragma unroll
+                for (int b = 0; b < 8; ++b) c[b] += hq[8 * lane + b];
+            }
+            uint32_t tot = 0;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) tot += c[b];
+            uint32_t incl = tot;   // keys in the digits of lanes >= this lane
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t x = __shfl_down_sync(0xffffffffu, incl, o);
+                if (lane + o < 32) incl += x;
+            }
+            const uint32_t above = incl - tot;
+            if (above < (uint32_t)krem && (uint32_t)krem <= incl) {
+                uint32_t acc = above;
+                int b = 7;
+                for (; b > 0; --b) {
+                    if (acc + c[b] >= (uint32_t)krem) break;
+                    acc += c[b];
+                }
+                lead->step[0] = 8 * lane + b;
+                lead->step[1] = acc;
+                lead->step[2] = acc + c[b] == (uint32_t)krem;   // the whole digit is taken
+            }
+        }
+        cl.sync();   // the digit is known
+        prefix = (prefix << width) | lead->step[0];
+        krem -= (int)lead->step[1];
+        const bool whole = lead->step[2] != 0;
+        top = shift;
+        if (stop_bits == 0 && top > 0 && whole) {
+            const uint32_t edge = lo + (prefix << top);
+            if (edge > 0) {
+                krem = 0;
+                return edge - 1;
+            }
+        }
+    }
+    return lo + (prefix << top);
+}
+
+// Grid: P CTAs per row (blockIdx.x = row * P + cluster rank), launched as clusters of P.
+// a.buf_cap: entries of each candidate buffer; chunk_words: bitmap words of the longest chunk.
+template <int NT>
+__global__ void __launch_bounds__(NT, 1) select_cluster_kernel(SelectArgs a, int P, int chunk_words)
+{
+    extern __shared__ __align__(16) uint8_t sel_smem[];
+    const int cap = a.buf_cap;
+    uint32_t* sample = reinterpret_cast<uint32_t*>(sel_smem);
+    uint64_t* cand = reinterpret_cast<uint64_t*>(sel_smem + a.sample_bytes);
+    uint64_t* gather = cand + cap;
+    uint32_t* gtmap = reinterpret_cast<uint32_t*>(gather + cap);
+    uint32_t* eqmap = gtmap + chunk_words;
+    __shared__ SelScalars<NT> sh;
+    __shared__ ClusterShared cs;
+    cg::cluster_group cl = cg::this_cluster();
+    const int p = (int)cl.block_rank();
+    ClusterShared* lead = cl.map_shared_rank(&cs, 0);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    grid_dep_wait();     // the scores come from the previous kernel
+    grid_dep_launch();
+
+    const int r = blockIdx.x / P;
+    const RowDesc rd = a.rows[r];
+    const int n = rd.ncols;
+    const int k = a.k;
+    const float* src = a.S + (int64_t)(a.src_from_list ? rd.list : r) * a.ld_s;
+    const int chunk = ((n + P - 1) / P + 127) & ~127;
+    const int c0 = min(n, p * chunk), c1 = min(n, c0 + chunk), nc = c1 - c0;
+    const int words = (nc + 31) >> 5;
+    if (n > k && nc > 0) prefetch_row_l2(src + c0, nc);
+    for (int w = tid; w < 2 * chunk_words; w += NT) gtmap[w] = 0;   // both bitmaps
+    if (tid == 0) {
+        sh.count = 0;
+        if (p == 0) {
+            cs.count = 0;
+            cs.overflow = 0;
+        }
+    }
+    cl.sync();   // the leader's counters are zero before any CTA adds to them
+
+    // ---- 1. tau from the row's sample, split among the CTAs by runs
+    uint32_t tau = 0;
+    if (n > k && n > cap) {
+        const int m = select_sample_size(n, k);
+        const uint32_t R = (uint32_t)(m / 32);
+        const uint32_t ra = R * (uint32_t)p / (uint32_t)P, rb = R * (uint32_t)(p + 1) / (uint32_t)P;
+        const int mine = (int)(rb - ra) * 32;
+        uint32_t lo = 0xffffffffu, hi = 0u;
+        for (int e = tid; e < mine; e += NT) {
+            const uint32_t run = ra + (uint32_t)(e >> 5);   // r n < 2^31
+            const int col = (int)(((run * (uint32_t)n) / R) & ~31u) + (e & 31);
+            const uint32_t u = score_key(__ldg(src + min(col, n - 1)));
+            sample[e] = u;
+            lo = min(lo, u);
+            hi = max(hi, u);
+        }
+        block_key_range<NT>(lo, hi, sh.scratch);   // also publishes the sample to the CTA
+        if (tid == 0) {
+            lead->lo[p] = lo;
+            lead->hi[p] = hi;
+        }
+        cl.sync();   // every CTA's range is in the leader
+        lo = 0xffffffffu;
+        hi = 0u;
+        for (int q = 0; q < P; ++q) {
+            lo = min(lo, lead->lo[q]);
+            hi = max(hi, lead->hi[q]);
+        }
+        const float expect = (float)k * m / n;
+        int rank = (int)ceilf(expect + 4.f * sqrtf(expect) + 4.f);
+        rank = min(rank, m);
+        tau = cluster_radix<NT>(cl, lead, P, [&](int i) { return sample[i]; }, mine, rank, lo, hi, 16, sh);
+    }
+
+    // ---- 2. this chunk's candidates; 3. into the leader's buffer
+    if (n > k) sel_append<NT>(src, c0, c1, tau, cand, cap, sh);
+    __syncthreads();
+    const uint32_t mine_c = sh.count;
+    if (tid == 0) {
+        uint32_t base = 0xffffffffu;
+        if (n > k) {
+            if (mine_c > (uint32_t)cap) atomicOr(&lead->overflow, 1u);
+            else if (mine_c > 0) base = atomicAdd(&lead->count, mine_c);
+        }
+        sh.base = base;
+    }
+    __syncthreads();
+    const uint32_t base = sh.base;
+    if (base != 0xffffffffu) {
+        if (base + mine_c <= (uint32_t)cap) {
+            uint64_t* g = cl.map_shared_rank(gather, 0);
+            for (uint32_t i = tid; i < mine_c; i += NT) g[base + i] = cand[i];
+        } else if (tid == 0) {
+            atomicOr(&lead->overflow, 1u);
+        }
+    }
+    cl.sync();   // the union is in the leader
+
+    // ---- the leader ranks the union (or the whole row)
+    if (p == 0) {
+        int krem = n;
+        uint32_t T = 0u, mode = 2u;   // rows of at most k columns: every column
+        if (n > k) {
+            const int count = (int)cs.count;
+            krem = k;
+            if (!cs.overflow && count >= k && count <= cap) {
+                uint32_t lo, hi;
+                sel_buf_keys<NT>(gather, count, lo, hi, sh);
+                T = radix_select_in<NT>([&](int i) { return (uint32_t)(gather[i] >> 32); }, count, krem, lo, hi,
+                                        sh.hist, sh.scratch);
+                mode = 0u;
+            } else {
+                T = radix_select<NT>([&](int i) { return score_key(__ldg(src + i)); }, n, krem, sh.hist,
+                                     sh.scratch);
+                mode = 1u;
+            }
+        }
+        if (tid == 0) {
+            cs.T = T;
+            cs.krem = krem;
+            cs.mode = mode;
+        }
+    }
+    cl.sync();   // T, krem and the mode are in the leader
+
+    // ---- 4. this chunk's marks
+    const uint32_t T = lead->T;
+    const int krem = lead->krem;
+    const uint32_t mode = lead->mode;
+    if (mode == 2u) {
+        for (int w = tid; w < words; w += NT) gtmap[w] = (w + 1) * 32 <= nc ? 0xffffffffu : ((1u << (nc & 31)) - 1u);
+    } else if (mode == 0u) {
+        for (uint32_t i = tid; i < mine_c; i += NT) {   // every key >= T of the chunk is a candidate here
+            const uint64_t e = cand[i];
+            const uint32_t u = score_key(__uint_as_float((uint32_t)(e >> 32)));
+            const uint32_t c = (uint32_t)e - (uint32_t)c0;
+            if (u > T) atomicOr(&gtmap[c >> 5], 1u << (c & 31));
+            else if (u == T) atomicOr(&eqmap[c >> 5], 1u << (c & 31));
+        }
+    } else {
+        for (int c = tid; c < nc; c += NT) {
+            const uint32_t u = score_key(__ldg(src + c0 + c));
+            if (u > T) atomicOr(&gtmap[c >> 5], 1u << (c & 31));
+            else if (u == T) atomicOr(&eqmap[c >> 5], 1u << (c & 31));
+        }
+    }
+    __syncthreads();
+    // thread-contiguous bitmap words; one block scan of the (> T, == T) counts
+    const int wpt = (words + NT - 1) / NT;
+    const int w0 = min(words, tid * wpt), w1 = min(words, w0 + wpt);
+    uint32_t ng = 0, ne = 0;
+    for (int w = w0; w < w1; ++w) {
+        ng += __popc(gtmap[w]);
+        ne += __popc(eqmap[w]);
+    }
+    const uint64_t own = ((uint64_t)ng << 32) | ne;
+    uint64_t incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+    }
+    uint64_t* wsum = reinterpret_cast<uint64_t*>(sh.hist);   // NT / 32 <= 32 entries
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    uint64_t before = incl - own, total = 0;
+    for (int w = 0; w < NT / 32; ++w) {
+        if (w < warp) before += wsum[w];
+        total += wsum[w];
+    }
+    const uint32_t G = (uint32_t)(total >> 32), E = (uint32_t)total;   // this chunk's > T and == T
+    if (tid == 0) {
+        lead->gt[p] = G;
+        lead->eq[p] = E;
+    }
+    cl.sync();   // every CTA's counts are in the leader
+    // this chunk's first output and its share of the T-ties (ties go to the lowest columns, so
+    // to the earlier chunks first)
+    uint32_t out0 = 0, ties_before = 0;
+    for (int q = 0; q < p; ++q) {
+        const uint32_t eq_q = lead->eq[q];
+        out0 += lead->gt[q] + min(eq_q, (uint32_t)max(0, krem - (int)ties_before));
+        ties_before += eq_q;
+    }
+    const uint32_t quota = min(E, (uint32_t)max(0, krem - (int)ties_before));
+    cl.sync();   // nothing reads the leader's shared memory after this
+
+    // ---- this chunk's columns, at out0 + (earlier threads' columns)
+    int32_t* oidx = a.out_idx + (int64_t)r * a.ld_idx;
+    float* osc = a.out_score ? a.out_score + (int64_t)r * a.ld_score : nullptr;
+    const int cnt = (int)(G + quota);
+    int32_t* stage = reinterpret_cast<int32_t*>(sel_smem);   // the sample and candidate buffer are free
+    const bool staged = (osc ? 2 * cnt : cnt) <= (a.sample_bytes + cap * 8) / 4;
+    const uint32_t g_before = (uint32_t)(before >> 32), e_before = (uint32_t)before;
+    uint32_t out = g_before + min(e_before, quota);
+    int left_e = (int)min(ne, (uint32_t)max(0, (int)quota - (int)e_before));
+    const int32_t* lrow = a.map.kind == kMapIdentity ? nullptr : a.map.list + (int64_t)rd.list * a.map.list_ld;
+    const bool per_word = a.map.kind == kMapIdentity || (a.map.kind == kMapBlocks && (a.map.block & 31) == 0);
+    __syncthreads();   // the candidates were read (marks) before the stage overwrites them
+    for (int w = w0; w < w1; ++w) {
+        uint32_t e = eqmap[w], te = 0;
+        for (; left_e > 0 && e; --left_e) {
+            const uint32_t low = e & (0u - e);
+            te |= low;
+            e ^= low;
+        }
+        uint32_t bits = gtmap[w] | te;
+        if (!bits) continue;
+        const int cw = c0 + w * 32;   // c0 is a multiple of 128
+        const int32_t wbase = a.map.kind == kMapIdentity ? cw + a.map.offset
+                              : per_word ? lrow[cw / a.map.block] * a.map.block + cw % a.map.block
+                                         : 0;
+        for (; bits; bits &= bits - 1) {
+            const int b = __ffs(bits) - 1;
+            const int col = cw + b;
+            const int32_t key = per_word ? wbase + b : a.map.kind == kMapList ? lrow[col] : map_col(a.map, rd, col);
+            const float sc = osc ? key_score(score_key(__ldg(src + col))) : 0.f;
+            if (staged) {
+                stage[out] = key;
+                if (osc) stage[cnt + out] = __float_as_int(sc);
+            } else {
+                oidx[out0 + out] = key;
+                if (osc) osc[out0 + out] = sc;
+            }
+            ++out;
+        }
+    }
+    if (staged) {
+        __syncthreads();
+        for (int j = tid; j < cnt; j += NT) {
+            oidx[out0 + j] = stage[j];
+            if (osc) osc[out0 + j] = __int_as_float(stage[cnt + j]);
+        }
+    }
+    if (p == 0) {   // padding past the row's columns
+        for (int j = min(n, k) + tid; j < k; j += NT) {
+            oidx[j] = -1;
+            if (osc) osc[j] = __int_as_float(0x7fc00000);
+        }
+    }
+}
+
+}  // namespace dsa

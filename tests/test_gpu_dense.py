@@ -128,13 +128,14 @@ def test_full_size_prefill_32k_sampled_rows():
     assert np.all(idx.max(1) <= np.arange(b.n_q))
 
 
-@pytest.mark.parametrize("n_rows", [2, 300])
+@pytest.mark.parametrize("n_rows", [2, 30, 300])
 @pytest.mark.parametrize("sampled_high", [True, False])
 def test_select_when_the_even_sample_misleads(sampled_high, n_rows):
     """The top-k picks a threshold from a sample of a long row: 2048 columns in 64 evenly spaced runs of
     32.  Keys that make exactly those columns score high (too few columns then pass the threshold) or
     low (too many pass) must still give the exact answer: integer inputs, compared exactly with the
-    oracle.  Two rows take the split select (several CTAs per row), 300 rows the one-CTA-per-row select."""
+    oracle.  Two rows take the split select (9 CTAs per row, sharing a global buffer), 30 rows the
+    cluster select (4 CTAs per row as one cluster), 300 rows the one-CTA-per-row select."""
     L, k = 20000, 3000
     b = workloads.ragged(30, [n_rows], [L], H=1, d=32, k=k, integer=True)
     starts = ((np.arange(64, dtype=np.int64) * L) // 64) & ~31        # the sample of a row of n = L
