@@ -299,10 +299,12 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
     dsa_status s;
     const int P = select_parts(n_rows, max_cols);
     if (sp.buf && sp.ctr && n_rows <= sp.max_rows && P > 1 && !n_rows_dev) {
-        // a row's CTAs as one cluster when they fit one (P <= 8) and its shared memory layout fits
+        // a row's CTAs as one cluster when they fit one (P <= 8), its shared memory layout fits and
+        // the rows are long: measured, 16 x 128K 31-33 -> 27-28 us, 16 x 32K unchanged, and HISA's
+        // ~8.4K-column token rows 3 us slower (ten cluster barriers against a short scan)
         const int chunk_words = ((((max_cols + P - 1) / P + 127) & ~127) + 31) / 32;
         const size_t csmem = cluster_smem_bytes(a.sample_bytes, a.buf_cap, chunk_words);
-        if (P <= kClusterMaxParts && csmem <= kSelectDynMax) {
+        if (P <= kClusterMaxParts && max_cols >= 16384 && csmem <= kSelectDynMax) {
             if ((s = set_smem(select_cluster_kernel<512>, csmem)) != DSA_OK) return s;
             DSA_LAUNCH(kProfSelect, st, launch_clustered(select_cluster_kernel<512>, n_rows * P, 512, csmem, P, st, a,
                                                          P, chunk_words));
