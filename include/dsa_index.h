@@ -250,9 +250,11 @@ dsa_status dsa_selftest_wait_timeout(uint32_t limit_us, void* ws, size_t ws_byte
  *    GPU that loads the library until the process exits.  A batch whose
  *    dsa_index_topk_workspace exceeds it is rejected with DSA_ERR_WORKSPACE
  *    before anything is launched.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *  - Every call looks up the array's device address in the current
+ *    device's context (cudaGetSymbolAddress, which allocates nothing), so a
+ *    context destroyed and made again (cudaDeviceReset) is followed.  The
+ *    first lookup on a device may load the library's device code: make the
+ *    first call on each device before any stream capture.
  *  - Every call on a device shares the one array: calls that overlap on the
  *    GPU (different streams, or different host threads) race and corrupt each
  *    other's results.  Serialise them.

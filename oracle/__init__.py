@@ -95,13 +95,14 @@ def dense(batch, rows=None, k=None, want_all=False, threads=None):
     return out
 
 
-def pair_scores(batch, rows, keys):
+def pair_scores(batch, rows, keys, threads=None):
     """Indexer score of each (query row, sequence-local key) pair, in fp64."""
     c = _Common(batch)
     rows, keys = _i32(rows), _i32(keys)
     out = np.empty(rows.size, np.float64)
     lib().orc_pair_scores(_p(c.Q), _p(c.K), _p(c.W), c.H, c.d, c.n_seqs, _p(c.q_off), _p(c.k_off),
-                          ctypes.c_int64(rows.size), _p(rows), _p(keys), _p(out))
+                          ctypes.c_int64(rows.size), _p(rows), _p(keys), _p(out),
+                          threads or default_threads())
     return out
 
 

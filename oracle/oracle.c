@@ -244,21 +244,43 @@ int orc_dense(const uint16_t* Q, const uint16_t* K, const float* W, int H, int d
     return 0;
 }
 
-/* Score arbitrary (query row, sequence-local key) pairs. */
-int orc_pair_scores(const uint16_t* Q, const uint16_t* K, const float* W, int H, int d,
-                    int n_seqs, const int32_t* q_off, const int32_t* k_off,
-                    int64_t n_pairs, const int32_t* rows, const int32_t* keys, double* out)
+/* Score arbitrary (query row, sequence-local key) pairs: key s of the query's
+ * own sequence, scored by the dense formula.  Pairs are independent; blocks
+ * of them run on `nthreads` threads. */
+typedef struct {
+    const uint16_t *Q, *K;
+    const float* W;
+    int H, d, n_seqs;
+    const int32_t *q_off, *k_off, *rows, *keys;
+    int64_t n_pairs;
+    double* out;
+} pairs_ctx;
+
+enum { PAIR_BLOCK = 1024 };
+
+static void pair_block(void* p, int64_t blk)
 {
-    double* q = (double*)malloc(sizeof(double) * ((size_t)H * d + H + d));
-    double* w = q + (size_t)H * d;
-    double* key = w + H;
-    for (int64_t p = 0; p < n_pairs; ++p) {
-        int b = seq_of_row(q_off, n_seqs, rows[p]);
-        load_query(Q, W, rows[p], H, d, q, w);
-        load_key(K, (int64_t)k_off[b] + keys[p], d, key);
-        out[p] = indexer_score(q, w, key, H, d);
+    pairs_ctx* c = (pairs_ctx*)p;
+    double* q = (double*)malloc(sizeof(double) * ((size_t)c->H * c->d + c->H + c->d));
+    double* w = q + (size_t)c->H * c->d;
+    double* key = w + c->H;
+    int64_t end = (blk + 1) * PAIR_BLOCK < c->n_pairs ? (blk + 1) * PAIR_BLOCK : c->n_pairs;
+    for (int64_t i = blk * PAIR_BLOCK; i < end; ++i) {
+        int b = seq_of_row(c->q_off, c->n_seqs, c->rows[i]);
+        load_query(c->Q, c->W, c->rows[i], c->H, c->d, q, w);
+        load_key(c->K, (int64_t)c->k_off[b] + c->keys[i], c->d, key);
+        c->out[i] = indexer_score(q, w, key, c->H, c->d);
     }
     free(q);
+}
+
+int orc_pair_scores(const uint16_t* Q, const uint16_t* K, const float* W, int H, int d,
+                    int n_seqs, const int32_t* q_off, const int32_t* k_off,
+                    int64_t n_pairs, const int32_t* rows, const int32_t* keys, double* out,
+                    int nthreads)
+{
+    pairs_ctx c = {Q, K, W, H, d, n_seqs, q_off, k_off, rows, keys, n_pairs, out};
+    parallel_rows(pair_block, &c, (n_pairs + PAIR_BLOCK - 1) / PAIR_BLOCK, nthreads);
     return 0;
 }
 

@@ -1307,24 +1307,16 @@ namespace {
 constexpr size_t kStaticScratchBytes = size_t(8) << 20;   // 8 MiB
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_static_scratch on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device with cudaGetSymbolAddress (with that device current) and cached.
+// Device address of g_static_scratch in the current device's context.  In host code the array's
+// name is only a host-side stand-in, so the address is looked up with cudaGetSymbolAddress (with
+// that device current) on every call: a cached address would go stale once the context is
+// destroyed and made again (cudaDeviceReset, or the primary context released and retained),
+// which loads the module again, possibly elsewhere.  The lookup allocates nothing.
 dsa_status static_scratch(void** out)
 {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
+    *out = p;
     return DSA_OK;
 }
 

@@ -118,7 +118,7 @@ def test_full_size_prefill_32k_sampled_rows():
     """Dense prefill T = L = 32K, H=64, d=128, k=2048: the whole batch on the GPU, sampled rows checked."""
     b = workloads.dense_prefill(seed=2)
     idx = Dev(b).topk(2048)
-    rows = workloads.stratified_rows(b.n_q, n_sample=40, head=8, tail=8)
+    rows = workloads.stratified_rows(b.n_q, n_sample=1024, head=16, tail=64)   # rows 0-15, the last 64, the rest spread
     ref = oracle.dense(b, rows=rows, k=2048, want_all=True)
     ascending_packed(idx[rows])
     check_tolerance_rows(idx[rows], ref["idx"], ref["all"])
@@ -159,10 +159,22 @@ def test_select_when_the_even_sample_misleads(sampled_high, n_rows):
     (42, [1] * 20, [5000 + 997 * i for i in range(20)], 512, "suffix"),
 ])
 def test_few_long_rows_exact(seed, q_lens, k_lens, k, mode):
-    """Few rows of many columns (decode): each row is ranked by several CTAs that share one candidate
-    buffer.  Integer inputs (many ties across the CTAs' column chunks), a row shorter than k, clamped
-    positions; exact against the oracle."""
+    """Few rows of many columns (decode): each row is ranked by several CTAs.  The first two cases
+    (6 and 4 rows: 9 and 14 CTAs per row, more than a cluster of 8) take the split select, whose CTAs
+    share one candidate buffer in global memory; the third (20 rows of up to ~24K columns: 7 CTAs
+    per row) takes the cluster select, whose CTAs meet in the leader's shared memory.  Integer
+    inputs (many ties across the CTAs' column chunks), a row shorter than k, clamped positions;
+    exact against the oracle."""
     exact_topk(workloads.ragged(seed, q_lens, k_lens, H=4, d=32, k=k, integer=True, pos_mode=mode), k)
+
+
+def test_cluster_select_short_rows_exact():
+    """The cluster select (20 single-query rows, the longest of 16K columns or more: 7 CTAs per row)
+    on rows that need no threshold: a row shorter than k (every column taken, -1 padding) and a row
+    with k < n <= the candidate buffer (the whole row goes into the buffer), beside long rows.
+    Integer inputs, exact against the oracle."""
+    k_lens = [300, 3000] + [16384 + 1231 * i for i in range(18)]
+    exact_topk(workloads.ragged(43, [1] * 20, k_lens, H=4, d=32, k=512, integer=True, pos_mode="suffix"), 512)
 
 
 @pytest.mark.parametrize("make", [

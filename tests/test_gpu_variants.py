@@ -195,7 +195,9 @@ def test_full_size_pivot_128k_sampled_groups():
     groups (early ones whose prefix is shorter than C, middle and last) checked against the oracle."""
     b = workloads.pivot_prefill(seed=3)
     G, C, k = 16, 8192, 2048
-    groups = [0, 3, 600, 4095, 8190, 8191]
+    # 64 groups: the first few (prefix shorter than C), 59 more spread evenly over the sequence, the last two
+    groups = sorted(set([0, 1, 3, 8190, 8191] + np.linspace(0, 8191, 61).astype(int).tolist()))
+    assert len(groups) >= 64
     dev = Dev(b)
     reuse = dev.pivot(k, G, C, 0)
     refine = dev.pivot(k, G, C, 1)

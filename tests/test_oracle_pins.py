@@ -373,3 +373,46 @@ def test_hisa_forced_blocks_and_external_kept():
         assert kept == sorted(kept)
     ext = oracle.hisa(b, B=128, keep=4, k=64, ext_kept=h["kept"])
     assert np.array_equal(ext["idx"], h["idx"])
+
+
+# ---------------------------------------------------------- pair scores
+
+def test_pair_scores_agree_with_dense_rows_across_sequences():
+    """oracle.pair_scores (the scorer behind the two-stage parity checks) returns, for arbitrary
+    (query row, sequence-local key) pairs of a ragged batch, exactly the dense oracle's score of
+    that entry (itself pinned above), including queries and keys of sequences after the first."""
+    b = workloads.ragged(71, [3, 4, 5], [7, 11, 9], H=4, d=32, k=5, integer=True, pos_mode="random")
+    res = oracle.dense(b, want_all=True)
+    rng = np.random.default_rng(5)
+    q_off = b.q_offsets.numpy()
+    rows, keys, expect = [], [], []
+    for t in range(b.n_q):
+        seq = int(np.searchsorted(q_off, t, side="right") - 1)
+        L = b.seq_lens()[seq]
+        elig = np.flatnonzero(np.isfinite(res["all"][t][:L]))
+        for s in rng.permutation(elig)[:4]:
+            rows.append(t)
+            keys.append(int(s))
+            expect.append(res["all"][t][s])
+    assert max(rows) >= q_off[2]                              # rows of the third sequence are covered
+    got = oracle.pair_scores(b, rows, keys)
+    assert np.array_equal(got, np.asarray(expect))
+
+
+def test_pair_scores_address_the_query_sequence_keys():
+    """Every key of sequence b is the constant vector (b + 1); every query is all ones with w = 1 on
+    one head: the score of any pair is (b + 1) * d, the sequence of the QUERY deciding which keys a
+    sequence-local index refers to.  A key read from another sequence, or rows and keys swapped,
+    gives a different value."""
+    d = 32
+    k_lens, q_lens = [5, 3, 6], [2, 3, 2]
+    K = np.concatenate([np.full((L, d), b + 1.0) for b, L in enumerate(k_lens)])
+    Q = np.ones((sum(q_lens), 1, d))
+    W = np.ones((sum(q_lens), 1))
+    pos = [4, 4, 2, 2, 2, 5, 5]
+    bt = make_batch(Q, K, W, q_lens, k_lens, pos)
+    rows = [0, 1, 2, 3, 4, 5, 6, 6]
+    keys = [4, 0, 2, 1, 0, 5, 0, 3]
+    seq_of_row = [0, 0, 1, 1, 1, 2, 2, 2]
+    got = oracle.pair_scores(bt, rows, keys)
+    assert got.tolist() == [(seq_of_row[r] + 1.0) * d for r in rows]
