@@ -276,7 +276,7 @@ def graph_times(step, steps, flush):
 def secondary(device, flush, steps, only=None, pivot_T=131072):
     out = {}
 
-    def run(name, make, extra, graph=False):
+    def run(name, make, extra, graph=False, post=None):
         if only and only not in name:
             return
         try:
@@ -298,6 +298,8 @@ def secondary(device, flush, steps, only=None, pivot_T=131072):
             step.dsa.profile_enable(False)
             r["kernels_us_per_step"] = {k: round(1e3 * v[0] / steps, 2) for k, v in prof.items()}
             r["launches_per_step"] = sum(v[1] for v in prof.values()) / steps
+            if post:
+                r.update(post(step, r["kernels_us_per_step"]))
             out[name] = r
             del step
             torch.cuda.empty_cache()
@@ -314,16 +316,69 @@ def secondary(device, flush, steps, only=None, pivot_T=131072):
         graph=True)
     run("dense_decode_B16_L131072_mtp2", lambda: DenseTopk(workloads.dense_decode(seed=1, L=131072), device),
         dec_extra, graph=True)
+    peaks = load_peaks()[0]
     if not only or "pivot" in only or "reuse" in only or "refine" in only:
         pv = workloads.pivot_prefill(seed=3, T=pivot_T)
         dense_pairs = pv.eligible_pairs()
         for mode, name in ((0, "reuse"), (1, "refine")):
             run(f"pivot_prefill_T{pivot_T}_G16_C8192_{name}", lambda m=mode: Pivot(pv, device, m),
-                lambda step, ms: {"dense_equiv_gpairs_s": round(dense_pairs / (ms * 1e-3) / 1e9, 2)})
+                lambda step, ms: {"dense_equiv_gpairs_s": round(dense_pairs / (ms * 1e-3) / 1e9, 2)},
+                post=lambda step, kus, m=mode: pivot_roofline(step.b, m, kus, peaks))
         del pv
-    run("hisa_decode_B4_L262144_keep64", lambda: Hisa(workloads.hisa_decode(seed=4), device), lambda s, ms: {},
-        graph=True)
+    run("hisa_decode_B4_L262144_keep64", lambda: Hisa(workloads.hisa_decode(seed=4), device),
+        lambda step, ms: hisa_bytes(step.b, ms, peaks), graph=True)
     return out
+
+
+def pivot_pairs(b):
+    """(proxy scan pairs, Refine pairs) of a PIVOT batch: the proxy of a group scans its sequence's
+    keys up to the group's last position; a query of Refine scores the group's candidates inside its
+    own prefix, at most min(C, its eligible keys) (exact to within G - 1 per query)."""
+    G, C = int(b.params["group"]), int(b.params["n_cand"])
+    qo, ko, pos = b.q_offsets.tolist(), b.k_offsets.tolist(), b.q_pos.tolist()
+    scan = refine = 0
+    for s in range(b.num_seqs):
+        L = ko[s + 1] - ko[s]
+        for g0 in range(qo[s], qo[s + 1], G):
+            g1 = min(g0 + G, qo[s + 1])
+            scan += min(L, max(pos[g0:g1]) + 1)
+            refine += sum(min(C, L, p + 1) for p in pos[g0:g1])
+    return scan, refine
+
+
+def pivot_roofline(b, mode, kernels_us, peaks):
+    """Tensor-pipe fraction of the PIVOT scoring launches (proxy scan; with Refine, also the gathered
+    candidate scoring), from their CUDA-event times: 2 H d flop per (row, key) pair against the
+    measured bf16 peak; the proxy top-C selection's bytes (each proxy score read once, C candidates
+    written per group) against the measured HBM copy bandwidth."""
+    scan, refine = pivot_pairs(b)
+    flop_pair = 2 * b.H * b.d
+    flops = (scan + (refine if mode == 1 else 0)) * flop_pair
+    t = kernels_us.get("score_tc", 0.0) * 1e-6
+    out = {"proxy_pairs": scan}
+    if mode == 1:
+        out["refine_pairs"] = refine
+    if t > 0:
+        tf = flops / t / 1e12
+        out["score_tflops"] = round(tf, 1)
+        out["score_frac_tensor"] = round(tf / peaks["bf16_tflops"], 4)
+    return out
+
+
+def hisa_bytes(b, ms, peaks):
+    """HBM bytes HISA must move per step: each sequence's pooled block keys (fp32, read once for its
+    queries), every query's kept blocks' keys (block 0, the `keep` best middle blocks and its own
+    block: at most (keep + 2) * B keys of d bf16), Q, W and the index rows; against the measured HBM
+    copy bandwidth (the step is latency-bound at this size)."""
+    B, keep, k = int(b.params["block"]), int(b.params["keep"]), int(b.params["k"])
+    pooled = sum((L + B - 1) // B for L in b.seq_lens()) * b.d * 4
+    kept = 0
+    for t in range(b.n_q):
+        n = int(b.q_pos[t]) + 1
+        kept += min(n, (keep + 2) * B) * b.d * 2
+    total = pooled + kept + b.Q.numel() * 2 + b.W.numel() * 4 + b.n_q * k * 4
+    gbs = total / (ms * 1e-3) / 1e9
+    return {"alg_bytes": total, "achieved_gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
 
 
 # ------------------------------------------------------------ baselines

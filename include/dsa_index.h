@@ -127,6 +127,41 @@ dsa_status dsa_index_topk(const dsa_batch* batch, const void* Q, const void* K, 
                           void* stream);
 
 /* --------------------------------------------------------------------
+ * Cross-layer index reuse: the selections of n_layers consecutive layers
+ * from fewer indexer runs.  Two schedules from the pages, combinable:
+ *  - retain_every = r (IndexCache, as the MLI abstract and the related-paper
+ *    list of the PIVOT page describe it: a few "full" layers run their own
+ *    indexer, the "shared" layers reuse the nearest full layer's top-k; a keep
+ *    ratio of 1/r): layer l's indexer runs only when l % r == 0; every other
+ *    layer reuses the selection of the nearest full layer below it.
+ *  - lag = 1 ("Multi-layer Indexer: overlapping selection and attention in
+ *    DeepSeek Sparse Attention", abstract): layer l attends over the selection
+ *    made for layer l - 1, so layer l's own indexer can run beside layer
+ *    l - 1's attention; layer 0 uses its own.  lag = 0: each layer uses the
+ *    selection of its own (nearest indexed) layer.
+ * dsa_index_layers_source(l, r, lag) is the layer whose indexer produces
+ * layer l's selection: r * floor((lag && l > 0 ? l - 1 : l) / r); -1 for a
+ * negative l, r < 1 or lag not 0/1.  Host-only.
+ * dsa_index_layers: Q, K, W and idx are HOST arrays of n_layers DEVICE
+ * pointers (layer l's inputs, laid out as for dsa_index_topk; every layer
+ * shares `batch`).  idx[l] [n_q, k] receives layer l's selection.  Each
+ * indexer run that some layer consumes is made by dsa_index_topk on
+ * `side_stream` (after the work already on `stream`), written into its first
+ * consumer's rows and copied to the others; runs nobody consumes are skipped.
+ * ready_events: NULL, or a HOST array of n_layers cudaEvent_t (created by the
+ * caller): event l is recorded on side_stream once idx[l] is complete, so the
+ * caller's work for layer l waits for that alone.  With NULL, `stream` waits
+ * for every selection before its later work.  The workspace is
+ * dsa_index_topk's (dsa_index_layers_workspace), reused by the runs in turn.
+ * side_stream must differ from stream.
+ */
+int32_t dsa_index_layers_source(int32_t layer, int32_t retain_every, int32_t lag);
+size_t dsa_index_layers_workspace(const dsa_batch* batch, int32_t k);
+dsa_status dsa_index_layers(const dsa_batch* batch, int32_t n_layers, const void* const* Q, const void* const* K,
+                            const float* const* W, int32_t k, int32_t retain_every, int32_t lag, int32_t* const* idx,
+                            void* const* ready_events, void* ws, size_t ws_bytes, void* stream, void* side_stream);
+
+/* --------------------------------------------------------------------
  * Dense top-k from host memory (no counterpart in the pages; the same
  * computation as dsa_index_topk for inputs that live in host memory).
  * Q, K, W, q_pos_host and idx are HOST pointers (page-locked for the copies

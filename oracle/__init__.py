@@ -170,3 +170,35 @@ def hisa(batch, B, keep, k, rows=None, pooled=None, ext_kept=None, threads=None)
                    _p(kept), _p(bs), ctypes.c_int64(max_blocks), _p(idx), _p(top),
                    threads or default_threads())
     return dict(kept=kept, block_scores=bs, idx=idx, top=top)
+
+
+def layer_sources(n_layers, retain_every, lag):
+    """For each of n_layers consecutive layers, the layer whose indexer made its selection, stepping
+    through the layers as the pages describe.  IndexCache (MLI abstract; related-paper list of the
+    PIVOT page): one layer in `retain_every` is "full" and runs its own indexer, starting with the
+    first; a "shared" layer reuses the top-k of the nearest full layer before it.  MLI (MLI
+    abstract), lag = 1: a layer attends over the selection the previous layer's indexer made, so its
+    own indexer can run beside its attention; the first layer has no predecessor and uses its own."""
+    src = []
+    last_full = None
+    prev_sel = None
+    for layer in range(n_layers):
+        if layer % retain_every == 0:
+            last_full = layer
+        own_sel = last_full                     # what this layer's (possibly reused) indexer provides
+        src.append(prev_sel if lag and layer > 0 else own_sel)
+        prev_sel = own_sel
+    return src
+
+
+def layer_topk(batches, k, retain_every, lag, threads=None):
+    """Selections of consecutive layers (one workloads.Batch per layer, same layout): the dense
+    top-k of each layer's source layer (layer_sources)."""
+    src = layer_sources(len(batches), retain_every, lag)
+    own = {}
+    out = []
+    for s in src:
+        if s not in own:
+            own[s] = dense(batches[s], k=k, threads=threads)["idx"]
+        out.append(own[s])
+    return out

@@ -8,8 +8,9 @@ pointers.  There is no CPU fallback: importing this package fails loudly
 when the compiled library is missing.
 
 Entry points mirror include/dsa_index.h:
-  index_scores, index_topk, pivot_group_index, hisa_pool_keys, hisa_index,
-  device_check, plus the *_workspace size queries.
+  index_scores, index_topk, index_topk_host, index_layers, pivot_group_index,
+  pivot_refine_candidates, hisa_pool_keys, hisa_index, device_check, plus the
+  *_workspace size queries.
 """
 from __future__ import annotations
 
@@ -19,7 +20,11 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdsaidx.so")
+# DSA_LIBRARY=checked loads the build whose kernels verify their device-side indices; every entry
+# point then also reads the workspace status word after its work (synchronising) and raises on a
+# recorded error.
+CHECKED = os.environ.get("DSA_LIBRARY", "") == "checked"
+LIB_PATH = os.path.join(_HERE, "libdsaidx_checked.so" if CHECKED else "libdsaidx.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python sparse_attention_indexer_04_b200/build.py` "
@@ -77,6 +82,10 @@ _sig("dsa_device_check", ctypes.c_int, _P, _P, ctypes.POINTER(ctypes.c_uint32))
 _sig("dsa_selftest_wait_timeout", ctypes.c_int, ctypes.c_uint32, _P, _SZ, _P)
 _sig("dsa_index_topk_static_capacity", _SZ)
 _sig("dsa_index_topk_static", ctypes.c_int, _B, _P, _P, _P, _I32, _P, _P, _P)
+_sig("dsa_index_layers_source", _I32, _I32, _I32, _I32)
+_sig("dsa_index_layers_workspace", _SZ, _B, _I32)
+_sig("dsa_index_layers", ctypes.c_int, _B, _I32, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P), _I32,
+     _I32, _I32, ctypes.POINTER(_P), ctypes.POINTER(_P), _P, _SZ, _P, _P)
 _sig("dsa_profile_enable", None, _I32)
 _sig("dsa_launch_count", ctypes.c_uint64)
 _sig("dsa_profile_kind_name", ctypes.c_char_p, _I32)
@@ -99,6 +108,20 @@ def _stream(stream=None):
 def _check(status: int, where: str):
     if status != 0:
         raise DsaError(status, where)
+
+
+ERR_BAD_INDEX = 4   # status-word code of the checked build: a device-side index outside its buffer
+
+
+def _after(ws, where: str, stream=None):
+    """Checked build only: wait for the call's work and raise if a kernel recorded an index error in
+    the workspace status word (other codes are left for device_check)."""
+    if not CHECKED:
+        return
+    torch.cuda.synchronize()   # every stream the call used
+    code, detail = (int(x) for x in ws[:8].view(torch.int32).cpu())
+    if code == ERR_BAD_INDEX:
+        raise DsaError(5, f"{where}: device index check failed at site {detail}")
 
 
 class Layout:
@@ -163,6 +186,7 @@ def index_scores(layout: Layout, Q, K, W, S=None, ws=None, stream=None):
     ws = _workspace(index_scores_workspace(layout), layout.device, ws)
     _check(_lib.dsa_index_scores(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), _ptr(S), S.stride(0), _ptr(ws),
                                  _bytes(ws), _stream(stream)), "dsa_index_scores")
+    _after(ws, "dsa_index_scores", stream)
     return S
 
 
@@ -179,7 +203,37 @@ def index_topk(layout: Layout, Q, K, W, k: int, idx=None, scores=None, want_scor
     ws = _workspace(index_topk_workspace(layout, k), layout.device, ws)
     _check(_lib.dsa_index_topk(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), k, _ptr(idx), _ptr(scores), _ptr(ws),
                                _bytes(ws), _stream(stream)), "dsa_index_topk")
+    _after(ws, "dsa_index_topk", stream)
     return (idx, scores) if want_scores else idx
+
+
+def index_layers_source(layer: int, retain_every: int, lag: int) -> int:
+    """The layer whose indexer run gives `layer` its selection (-1 for invalid arguments)."""
+    return int(_lib.dsa_index_layers_source(layer, retain_every, lag))
+
+
+def index_layers(layout: Layout, Qs, Ks, Ws, k: int, retain_every: int = 1, lag: int = 0, idx=None, events=None,
+                 ws=None, stream=None, side_stream=None):
+    """Selections of len(Qs) layers (dsa_index_layers): idx[l] [n_q, k] int32 for layer l.  `events`: optional
+    torch.cuda.Event per layer, recorded once idx[l] is complete (then `stream` is not made to wait)."""
+    n = len(Qs)
+    if not (len(Ks) == len(Ws) == n):
+        raise ValueError("one Q, K and W per layer")
+    if idx is None:
+        idx = [torch.empty(layout.num_queries, k, dtype=torch.int32, device=layout.device) for _ in range(n)]
+    if side_stream is None:
+        raise ValueError("index_layers needs a side stream distinct from the compute stream")
+    arr = lambda ts: (_P * n)(*[t.data_ptr() for t in ts])
+    ev = None
+    if events is not None:
+        for e in events:
+            e.record(stream if stream is not None else torch.cuda.current_stream())   # creates the event
+        ev = (_P * n)(*[e.cuda_event for e in events])
+    ws = _workspace(int(_lib.dsa_index_layers_workspace(layout.ref(), k)), layout.device, ws)
+    _check(_lib.dsa_index_layers(layout.ref(), n, arr(Qs), arr(Ks), arr(Ws), k, retain_every, lag, arr(idx), ev,
+                                 _ptr(ws), _bytes(ws), _stream(stream), _stream(side_stream)), "dsa_index_layers")
+    _after(ws, "dsa_index_layers", stream)
+    return idx
 
 
 def index_topk_host_workspace(layout: Layout, k: int) -> int:
@@ -198,6 +252,7 @@ def index_topk_host(layout: Layout, q_pos, Q, K, W, k: int, idx, ws, stream=None
     _check(_lib.dsa_index_topk_host(layout.ref(), _ptr(q_pos), _ptr(Q), _ptr(K), _ptr(W), k, _ptr(idx), _ptr(ws),
                                     _bytes(ws), _stream(stream), _stream(in_stream), _stream(out_stream)),
            "dsa_index_topk_host")
+    _after(ws, "dsa_index_topk_host", stream)
     return idx
 
 
@@ -237,6 +292,7 @@ def pivot_group_index(layout: Layout, Q, K, W, k: int, group: int, n_cand: int, 
     ws = _workspace(pivot_group_index_workspace(layout, k, group, n_cand, mode), layout.device, ws)
     _check(_lib.pivot_group_index(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), k, group, n_cand, mode, _ptr(idx),
                                   _ptr(cand), _ptr(ws), _bytes(ws), _stream(stream)), "pivot_group_index")
+    _after(ws, "pivot_group_index", stream)
     return (idx, cand) if want_cand else idx
 
 
@@ -252,6 +308,7 @@ def pivot_refine_candidates(layout: Layout, Q, K, W, k: int, group: int, cand, i
     ws = _workspace(pivot_refine_candidates_workspace(layout, k, group, n_cand), layout.device, ws)
     _check(_lib.pivot_refine_candidates(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), k, group, n_cand, _ptr(cand),
                                         _ptr(idx), _ptr(ws), _bytes(ws), _stream(stream)), "pivot_refine_candidates")
+    _after(ws, "pivot_refine_candidates", stream)
     return idx
 
 
@@ -284,6 +341,7 @@ def hisa_index(layout: Layout, Q, K, W, pooled, k: int, block: int, keep: int, i
     ws = _workspace(hisa_index_workspace(layout, k, block, keep), layout.device, ws)
     _check(_lib.hisa_index(layout.ref(), _ptr(Q), _ptr(K), _ptr(W), _ptr(pooled), k, block, keep, _ptr(idx),
                            _ptr(kept), _ptr(ws), _bytes(ws), _stream(stream)), "hisa_index")
+    _after(ws, "hisa_index", stream)
     return (idx, kept) if want_kept else idx
 
 

@@ -1,4 +1,12 @@
-"""Build libdsaidx.so in-tree with nvcc for sm_100a (cross-compiles without a GPU)."""
+"""Build libdsaidx.so in-tree with nvcc for sm_100a (cross-compiles without a GPU).
+
+Two builds of the same sources: libdsaidx.so, and libdsaidx_checked.so compiled with
+-DDSA_DEVICE_CHECKS=1, whose kernels verify the indices they compute on the device (gathered key
+rows, candidate positions, bitmap words, output slots) and record a violation in the workspace
+status word instead of touching memory outside a buffer.  The checked build is for debugging and
+for the test that runs the exact parity cases through it; the package loads it when the
+environment variable DSA_LIBRARY is "checked".
+"""
 import glob
 import os
 import subprocess
@@ -8,6 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libdsaidx.so")
+LIB_CHECKED = os.path.join(HERE, "libdsaidx_checked.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -26,22 +35,35 @@ def deps():
         sorted(glob.glob(os.path.join(INCLUDE, "*.h"))) + [os.path.abspath(__file__)]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib=LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and up_to_date():
-        return LIB
+def _command(lib, extra):
     nvcc = os.environ.get("NVCC", "nvcc")
-    cmd = [nvcc, *NVCC_FLAGS, *extra, "-I", INCLUDE, "-o", LIB + ".tmp", *sources()]
-    if verbose:
-        print(" ".join(cmd))
-    subprocess.check_call(cmd)
-    os.replace(LIB + ".tmp", LIB)
+    return [nvcc, *NVCC_FLAGS, *extra, "-I", INCLUDE, "-o", lib + ".tmp", *sources()]
+
+
+def build(force: bool = False, verbose: bool = False, extra=(), checked: bool = True) -> str:
+    """Builds libdsaidx.so (and, with `checked`, libdsaidx_checked.so; the two compile in parallel)."""
+    jobs = []
+    if force or not up_to_date(LIB):
+        jobs.append((LIB, list(extra)))
+    if checked and (force or not up_to_date(LIB_CHECKED)):
+        jobs.append((LIB_CHECKED, list(extra) + ["-DDSA_DEVICE_CHECKS=1"]))
+    procs = []
+    for lib, ex in jobs:
+        cmd = _command(lib, ex)
+        if verbose:
+            print(" ".join(cmd))
+        procs.append((lib, subprocess.Popen(cmd)))
+    for lib, p in procs:
+        if p.wait() != 0:
+            raise subprocess.CalledProcessError(p.returncode, _command(lib, []))
+        os.replace(lib + ".tmp", lib)
     return LIB
 
 

@@ -94,6 +94,10 @@ dsa_status check_ws(void* ws, size_t ws_bytes, size_t need)
     return DSA_OK;
 }
 
+// The status word of the entry point running on this host thread: select launches hand it to their
+// kernels (checked builds record index errors there).  Set by every entry point before its launches.
+thread_local uint32_t* g_status = nullptr;
+
 dsa_status launched()
 {
     return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
@@ -289,6 +293,7 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
     if (n_rows <= 0) return DSA_OK;
     SelectArgs a{};
     a.rows = rows; a.n_rows = n_rows; a.k = k; a.map = map; a.S = S; a.ld_s = ld_s;
+    a.status = g_status;
     a.src_from_list = src_from_list ? 1 : 0;
     a.out_idx = out_idx; a.ld_idx = ld_idx; a.out_score = out_score; a.ld_score = ld_score;
     a.n_rows_dev = n_rows_dev;
@@ -487,7 +492,8 @@ dsa_status launch_tc_d(int H, const CUtensorMap& mq, const CUtensorMap& mk, cons
 // map(c) of the row's sequence.
 dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const TcSource& src, int H, int D,
                     const void* K, int64_t n_k, const int32_t* k_base, const ColMap& map, int32_t max_cols, float* S,
-                    int64_t ld, TcUnit* units, int32_t* tile_base, uint32_t* status, cudaStream_t st)
+                    int64_t ld, TcUnit* units, int32_t* tile_base, uint32_t* status, cudaStream_t st,
+                    bool units_ready = false)
 {
     if (n_rows <= 0 || max_cols <= 0 || n_k <= 0) return DSA_OK;
     const int32_t TQ = tc_tile_rows(H);
@@ -499,11 +505,13 @@ dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const
     if (!make_tile_map(&mq, src.Q, src.q_rows * H, D, 256) || !make_tile_map(&mk, K, n_k, D, 128) ||
         !make_tile_map(&mkg, K, n_k, D, 1))
         return DSA_ERR_CUDA;
-    DSA_LAUNCH(kProfSetup, st, launch_pdl(latency_bound(int64_t(tiles) * splits), tc_units_kernel, 1, 1024, 0, st, rows,
-                                          n_rows, row_base, src.seq_off, src.n_seqs, TQ, splits, k_base, tile_base,
-                                          units));
-    dsa_status s = launched();
-    if (s != DSA_OK) return s;
+    if (!units_ready) {   // (else dense_setup_kernel wrote them)
+        DSA_LAUNCH(kProfSetup, st, launch_pdl(latency_bound(int64_t(tiles) * splits), tc_units_kernel, 1, 1024, 0, st,
+                                              rows, n_rows, row_base, src.seq_off, src.n_seqs, TQ, splits, k_base,
+                                              tile_base, units));
+        dsa_status s = launched();
+        if (s != DSA_OK) return s;
+    }
     int32_t max_q = 0;
     for (int b = 0; b < src.n_seqs; ++b) max_q = std::max(max_q, src.seq_off_host[b + 1] - src.seq_off_host[b]);
     const int n_acc = std::min(max_q, TQ) > TQ / 2 ? 2 : 1;
@@ -519,6 +527,7 @@ dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const
     a.S = S;
     a.ld_s = ld;
     a.status = status;
+    a.n_keys = n_k;
     switch (D) {
     case 32: return launch_tc_d<32>(H, mq, mk, mkg, a, tiles * splits, n_acc, st);
     case 64: return launch_tc_d<64>(H, mq, mk, mkg, a, tiles * splits, n_acc, st);
@@ -779,7 +788,50 @@ size_t hisa_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, 
 
 dsa_status clear_status(void* ws, cudaStream_t st)
 {
+    g_status = static_cast<uint32_t*>(ws);
     return cudaMemsetAsync(ws, 0, kHeaderBytes, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// dsa_index_topk for a batch scored in one launch (decode; prefill within the score buffer): one
+// set-up kernel (the header cleared, rows, work units), the scoring launch, the select: three
+// launches, the later two programmatic where their grids are small.
+dsa_status dense_topk_one_launch(const dsa_batch* b, const HostInfo& hi, const TcSource& src, const void* K,
+                                 int32_t k, int32_t* idx, float* scores, const DensePlan& p, void* ws,
+                                 cudaStream_t st)
+{
+    static_assert(kHeaderBytes % 4 == 0, "header words");
+    const int32_t TQ = tc_tile_rows(b->num_heads);
+    g_status = static_cast<uint32_t*>(ws);
+    DenseSetupArgs a{};
+    a.q_off = b->q_offsets;
+    a.k_off = b->k_offsets;
+    a.q_pos = b->q_pos;
+    a.rows = p.rows;
+    a.units = p.units;
+    a.header = static_cast<uint32_t*>(ws);
+    a.header_words = (int32_t)(kHeaderBytes / 4);
+    a.n_seqs = b->num_seqs;
+    a.n_q = b->num_queries;
+    a.TQ = TQ;
+    int32_t tiles = 0;
+    for (int i = 0; i < b->num_seqs; ++i) {
+        a.tile_base[i] = tiles;
+        tiles += (b->q_offsets_host[i + 1] - b->q_offsets_host[i] + TQ - 1) / TQ;
+    }
+    a.tile_base[b->num_seqs] = tiles;
+    a.splits = tc_splits(tiles, hi.max_k);   // as tc_score derives it
+    a.n_units = tiles * a.splits;
+    const int grid = (std::max(a.n_q, a.n_units) + 255) / 256;
+    // a plain launch: it starts once the stream's earlier work (which may use this workspace) is done
+    DSA_LAUNCH(kProfSetup, st, launch_pdl(false, dense_setup_kernel, grid, 256, 0, st, a));
+    dsa_status s = launched();
+    if (s != DSA_OK) return s;
+    const int64_t ld = score_ld(hi.max_k);
+    uint32_t* status = static_cast<uint32_t*>(ws);
+    s = tc_score(p.rows, b->num_queries, 0, src, b->num_heads, b->head_dim, K, b->num_keys, b->k_offsets, ColMap{},
+                 hi.max_k, p.S, ld, p.units, p.tile_base, status, st, true);
+    if (s != DSA_OK) return s;
+    return launch_select(p.rows, b->num_queries, hi.max_k, k, ColMap{}, p.S, ld, false, idx, k, scores, k, st, p.split);
 }
 
 // PIVOT Refine's second stage: each query scores its eligible candidates (query_rows, list map m)
@@ -875,15 +927,81 @@ dsa_status dsa_index_topk(const dsa_batch* b, const void* Q, const void* K, cons
     if ((s = check_ws(ws, ws_bytes, dense_plan(nullptr, b, hi, k, &p))) != DSA_OK) return s;
     dense_plan(static_cast<char*>(ws), b, hi, k, &p);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const TcSource src{Q, b->num_queries, W, b->q_offsets, b->q_offsets_host, b->num_seqs};
+    if (b->num_queries > 0 && b->num_keys > 0 && hi.max_k > 0 && b->num_seqs <= kSetupMaxSeqs &&
+        chunk_rows(b->num_queries, score_ld(hi.max_k)) >= b->num_queries)
+        return dense_topk_one_launch(b, hi, src, K, k, idx, scores, p, ws, st);
     if ((s = clear_status(ws, st)) != DSA_OK) return s;
     if (b->num_queries == 0) return DSA_OK;
     DSA_LAUNCH(kProfSetup, st, dense_rows_kernel<<<(b->num_queries + 255) / 256, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos,
                                                                     b->num_seqs, b->num_queries, p.rows));
     if ((s = launched()) != DSA_OK) return s;
-    const TcSource src{Q, b->num_queries, W, b->q_offsets, b->q_offsets_host, b->num_seqs};
     return tc_score_and_select(p.rows, b->num_queries, src, b->num_heads, b->head_dim, K, b->num_keys, b->k_offsets,
                                ColMap{}, hi.max_k, p.S, p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, scores, st,
                                p.split);
+}
+
+// ------------------------------------------------- cross-layer index reuse
+int32_t dsa_index_layers_source(int32_t layer, int32_t retain_every, int32_t lag)
+{
+    if (layer < 0 || retain_every < 1 || (lag != 0 && lag != 1)) return -1;
+    const int32_t consumer = lag == 1 && layer > 0 ? layer - 1 : layer;   // MLI: the previous layer's selection
+    return consumer / retain_every * retain_every;                       // IndexCache: its nearest indexed layer
+}
+
+size_t dsa_index_layers_workspace(const dsa_batch* b, int32_t k) { return dsa_index_topk_workspace(b, k); }
+
+dsa_status dsa_index_layers(const dsa_batch* b, int32_t n_layers, const void* const* Q, const void* const* K,
+                            const float* const* W, int32_t k, int32_t retain_every, int32_t lag, int32_t* const* idx,
+                            void* const* ready_events, void* ws, size_t ws_bytes, void* stream, void* side_stream)
+{
+    if (n_layers < 1 || retain_every < 1 || (lag != 0 && lag != 1) || !Q || !K || !W || !idx) return DSA_ERR_INVALID_ARG;
+    if (!side_stream || side_stream == stream) return DSA_ERR_INVALID_ARG;
+    HostInfo hi;
+    dsa_status s = check_batch(b, &hi);
+    if (s != DSA_OK) return s;
+    for (int32_t l = 0; l < n_layers; ++l) {
+        if (!idx[l]) return DSA_ERR_INVALID_ARG;
+        if ((s = check_tensors(b, Q[l], K[l], W[l])) != DSA_OK) return s;
+    }
+    if (k < 1 || k > kMaxK || !select_fits(k, hi.max_k)) return DSA_ERR_UNSUPPORTED;
+    if ((s = check_ws(ws, ws_bytes, dsa_index_topk_workspace(b, k))) != DSA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream), side = static_cast<cudaStream_t>(side_stream);
+    cudaEvent_t ev_in, ev_out;
+    if (cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&ev_out, cudaEventDisableTiming) != cudaSuccess) {
+        cudaEventDestroy(ev_in);
+        return DSA_ERR_CUDA;
+    }
+    bool ok = true;
+    auto chk = [&](cudaError_t e) { ok = ok && e == cudaSuccess; };
+    // the side stream starts after the work already on `stream` (the layers' inputs)
+    chk(cudaEventRecord(ev_in, st));
+    chk(cudaStreamWaitEvent(side, ev_in, 0));
+    const size_t row_bytes = size_t(std::max(b->num_queries, 0)) * k * sizeof(int32_t);
+    // each indexed layer's top-k, written into its first consumer's rows and copied to the others
+    for (int32_t f = 0; f < n_layers && ok && s == DSA_OK; f += retain_every) {
+        int32_t first = -1;
+        for (int32_t l = 0; l < n_layers; ++l) {
+            if (dsa_index_layers_source(l, retain_every, lag) != f) continue;
+            if (first < 0) {
+                first = l;
+                s = dsa_index_topk(b, Q[f], K[f], W[f], k, idx[l], nullptr, ws, ws_bytes, side);
+                if (s != DSA_OK) break;
+            } else if (row_bytes > 0) {
+                chk(cudaMemcpyAsync(idx[l], idx[first], row_bytes, cudaMemcpyDeviceToDevice, side));
+            }
+            if (ready_events && ready_events[l]) chk(cudaEventRecord(static_cast<cudaEvent_t>(ready_events[l]), side));
+        }
+    }
+    if (!ready_events) {   // without per-layer events, `stream` waits for every selection
+        chk(cudaEventRecord(ev_out, side));
+        chk(cudaStreamWaitEvent(st, ev_out, 0));
+    }
+    cudaEventDestroy(ev_in);
+    cudaEventDestroy(ev_out);
+    if (s != DSA_OK) return s;
+    return ok ? DSA_OK : DSA_ERR_CUDA;
 }
 
 // ------------------------------------------------- dense top-k from host memory
@@ -1087,6 +1205,7 @@ dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, c
         ra.groups = p.groups; ra.query_rows = p.query_rows; ra.cand_rows = p.cand_rows;
         ra.gsel = p.gsel; ra.gscore = p.gscore; ra.kp = kp; ra.k = k; ra.cand = cand; ra.C = C;
         ra.idx = idx; ra.ld_idx = k; ra.fb_rows = p.fb_rows; ra.fb_count = reuse_fallback_count(ws);
+        ra.status = static_cast<uint32_t*>(ws);
         const size_t smem = reuse_smem_bytes(kp);
         if ((s = set_smem(pivot_reuse_kernel, smem)) != DSA_OK) return s;
         DSA_LAUNCH(kProfSelect, st, pivot_reuse_kernel<<<ng, kReuseThreads, smem, st>>>(ra));

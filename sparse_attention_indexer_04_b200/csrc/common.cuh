@@ -16,13 +16,34 @@ enum : uint32_t {
     kErrNone = 0,
     kErrWaitTimeout = 1,   // a bounded wait on an mbarrier ran out
     kErrBadRow = 2,        // a row descriptor points outside its buffers
+    kErrBadIndex = 4,      // (checked builds) an index computed on the device fell outside its buffer
 };
 
 __device__ __forceinline__ void record_error(uint32_t* status, uint32_t code, uint32_t detail)
 {
+    if (!status) return;
     if (atomicCAS(status, 0u, code) == 0u)
         status[1] = detail;
 }
+
+// Checked builds (compiled with -DDSA_DEVICE_CHECKS=1): DSA_CHECK(ok, status, where) is `ok`, and a
+// false `ok` records kErrBadIndex with detail `where` in the status word, so the caller can skip the
+// access it guards.  Otherwise it is `true` and costs nothing.  Every guarded index is in range by
+// construction; the checks exist to catch a broken invariant (a gathered key row, a candidate
+// position, a bitmap word, an output slot) without a memory fault.
+#ifndef DSA_DEVICE_CHECKS
+#define DSA_DEVICE_CHECKS 0
+#endif
+__device__ __forceinline__ bool check_index(bool ok, uint32_t* status, uint32_t where)
+{
+    if (!ok) record_error(status, kErrBadIndex, where);
+    return ok;
+}
+#if DSA_DEVICE_CHECKS
+#define DSA_CHECK(ok, status, where) (::dsa::check_index((ok), (status), (where)))
+#else
+#define DSA_CHECK(ok, status, where) (true)
+#endif
 
 // -------------------------------------------------------- score ordering
 // Order-preserving map of an fp32 score to uint32: a larger score gives a

@@ -44,6 +44,7 @@ struct ReuseArgs {
     int64_t ld_idx;
     RowDesc* fb_rows;            // queries left to the per-query selection
     int32_t* fb_count;
+    uint32_t* status;            // the workspace status word (checked builds record index errors there)
 };
 
 constexpr int kReuseThreads = 256;
@@ -102,7 +103,10 @@ __global__ void __launch_bounds__(kReuseThreads) pivot_reuse_kernel(ReuseArgs a)
         for (int w = 0; w < warp; ++w) before += sh.hist[w];
         for (int i = i0; i < i1; ++i) {
             const bool is_tie = key[i] == T;
-            if (key[i] < T || (is_tie && before >= (uint32_t)krem)) tail[atomicAdd(&s_tail_n, 1u)] = i;
+            if (key[i] < T || (is_tie && before >= (uint32_t)krem)) {
+                const uint32_t e = atomicAdd(&s_tail_n, 1u);
+                if (DSA_CHECK(e < (uint32_t)kReuseMaxTail, a.status, 401)) tail[e] = i;   // the tail holds <= kp - k
+            }
             before += is_tie;
         }
         __syncthreads();
@@ -173,6 +177,7 @@ __global__ void __launch_bounds__(kReuseThreads) pivot_reuse_kernel(ReuseArgs a)
                     if (drop_pos[mid] < i) lo = mid + 1; else hi = mid;
                 }
                 if (lo < drop && drop_pos[lo] == i) continue;
+                if (!DSA_CHECK(i - lo < k && col[i] >= 0 && col[i] < a.C, a.status, 402)) continue;
                 o[i - lo] = cl[col[i]];
             }
             for (int i = m - drop + tid; i < k; i += NT) o[i] = -1;

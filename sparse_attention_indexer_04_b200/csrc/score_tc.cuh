@@ -53,6 +53,7 @@ struct TcArgs {
     uint32_t* status;
     int32_t n_stages;
     int32_t pad_;
+    int64_t n_keys;          // rows of K (checked builds verify every gathered key row against it)
 };
 
 template <int D, int H>
@@ -213,6 +214,9 @@ __global__ void __launch_bounds__(GATHER ? kTcThreads : kTcThreadsTiles, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) y[e] = krow0 + map_col(a.map, first, c0 + e < ncmax ? c0 + e : 0);
             }
+#pragma unroll
+            for (int e = 0; e < 4; ++e)   // a gathered key row of K (an out-of-range row would read zeros)
+                if (!DSA_CHECK(y[e] >= 0 && y[e] < a.n_keys, a.status, 101)) y[e] = 0;
         };
         // Keys other units read again stay in L2 while the score rows stream out.
         const uint64_t keep_keys = l2_policy_evict_last();

@@ -68,6 +68,7 @@ struct SelectArgs {
     const int32_t* n_rows_dev;   // nullable: rows [*n_rows_dev, n_rows) are skipped (a count a kernel wrote)
     int32_t out_from_qrow;       // 1: row r writes output row rows[r].qrow instead of r
     int32_t pad_;
+    uint32_t* status;            // the workspace status word (checked builds record index errors there)
 };
 
 
@@ -370,7 +371,8 @@ __device__ __forceinline__ void sel_buf_keys(uint64_t* buf, int count, uint32_t&
 // sample) by radix passes over the whole row.
 template <int NT>
 __device__ __forceinline__ void sel_mark(const float* src, int n, int k, uint64_t* buf, int count, int cap,
-                                         int& krem, uint32_t* gtmap, uint32_t* eqmap, SelScalars<NT>& sh)
+                                         int& krem, uint32_t* gtmap, uint32_t* eqmap, SelScalars<NT>& sh,
+                                         uint32_t* status = nullptr)
 {
     const int tid = threadIdx.x;
     krem = k;
@@ -381,6 +383,7 @@ __device__ __forceinline__ void sel_mark(const float* src, int n, int k, uint64_
                                                     lo, hi, sh.hist, sh.scratch);
         for (int i = tid; i < count; i += NT) {
             const uint32_t u = (uint32_t)(buf[i] >> 32), c = (uint32_t)buf[i];
+            if (!DSA_CHECK(c < (uint32_t)n, status, 201)) continue;   // a candidate column of the row
             if (u > thresh) atomicOr(&gtmap[c >> 5], 1u << (c & 31));
             else if (u == thresh) atomicOr(&eqmap[c >> 5], 1u << (c & 31));
         }
@@ -463,6 +466,7 @@ __device__ __forceinline__ void sel_emit(const SelectArgs& a, const RowDesc& rd,
             const int col = c0 + b;
             const int32_t key = per_word ? wbase + b : a.map.kind == kMapList ? lrow[col] : map_col(a.map, rd, col);
             const float sc = osc ? key_score(score_key(__ldg(src + col))) : 0.f;
+            if (!DSA_CHECK(out < (uint32_t)k && key >= 0, a.status, 202)) { ++out; continue; }   // output slot, key
             if (staged) {
                 stage[out] = key;
                 if (osc) stage[k + out] = __float_as_int(sc);
@@ -544,7 +548,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_stream_kernel(SelectArgs
         __syncthreads();
         sel_append<NT>(src, 0, n, tau, buf, cap, sh);
         __syncthreads();
-        sel_mark<NT>(src, n, k, buf, (int)sh.count, cap, krem, gtmap, eqmap, sh);
+        sel_mark<NT>(src, n, k, buf, (int)sh.count, cap, krem, gtmap, eqmap, sh, a.status);
     } else {
         __syncthreads();
         sel_mark_all<NT>(n, gtmap);
@@ -618,7 +622,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_split_kernel(SelectArgs 
         if (count >= k && count <= cap)
             for (int i = tid; i < count; i += NT) buf[i] = __ldcg(reinterpret_cast<const unsigned long long*>(g) + i);
         __syncthreads();
-        sel_mark<NT>(src, n, k, buf, count, cap, krem, gtmap, eqmap, sh);
+        sel_mark<NT>(src, n, k, buf, count, cap, krem, gtmap, eqmap, sh, a.status);
     } else {
         sel_mark_all<NT>(n, gtmap);
     }

@@ -252,6 +252,7 @@ __global__ void __launch_bounds__(NT, 1) select_cluster_kernel(SelectArgs a, int
             const uint64_t e = cand[i];
             const uint32_t u = score_key(__uint_as_float((uint32_t)(e >> 32)));
             const uint32_t c = (uint32_t)e - (uint32_t)c0;
+            if (!DSA_CHECK(c < (uint32_t)nc, a.status, 301)) continue;   // a column of this CTA's chunk
             if (u > T) atomicOr(&gtmap[c >> 5], 1u << (c & 31));
             else if (u == T) atomicOr(&eqmap[c >> 5], 1u << (c & 31));
         }
@@ -333,6 +334,10 @@ __global__ void __launch_bounds__(NT, 1) select_cluster_kernel(SelectArgs a, int
             const int col = cw + b;
             const int32_t key = per_word ? wbase + b : a.map.kind == kMapList ? lrow[col] : map_col(a.map, rd, col);
             const float sc = osc ? key_score(score_key(__ldg(src + col))) : 0.f;
+            if (!DSA_CHECK(out0 + out < (uint32_t)k && out < (uint32_t)cnt && key >= 0, a.status, 302)) {
+                ++out;
+                continue;
+            }
             if (staged) {
                 stage[out] = key;
                 if (osc) stage[cnt + out] = __float_as_int(sc);

@@ -19,6 +19,60 @@ __global__ void dense_rows_kernel(const int32_t* q_off, const int32_t* k_off, co
     rows[t] = RowDesc{t, b, eligible_count(q_pos[t], k_off[b + 1] - k_off[b]), 0};
 }
 
+// Dense top-k set-up in one launch, for a batch scored in one tensor-core launch (no row chunks):
+// the workspace header cleared, one row per query (as dense_rows_kernel) and the launch's work
+// units (as tc_units_kernel), each unit computed alone from the segments' tile offsets, which the
+// host knows from the query offsets and passes in.  The units' key ranges come from the queries'
+// positions directly, so the kernel does not wait on its own rows.
+constexpr int kSetupMaxSeqs = 480;   // sequences whose tile offsets fit in the argument block
+
+struct DenseSetupArgs {
+    const int32_t* q_off;
+    const int32_t* k_off;
+    const int32_t* q_pos;
+    RowDesc* rows;
+    TcUnit* units;
+    uint32_t* header;        // zeroed: header_words words
+    int32_t header_words;
+    int32_t n_seqs;
+    int32_t n_q;
+    int32_t TQ;              // query rows per tile
+    int32_t splits;          // key-range parts per tile
+    int32_t n_units;         // tile_base[n_seqs] * splits
+    int32_t tile_base[kSetupMaxSeqs + 1];   // first tile of each sequence (tiles cut per sequence)
+};
+
+__global__ void dense_setup_kernel(const __grid_constant__ DenseSetupArgs a)
+{
+    grid_dep_launch();   // the scoring kernel may set up; it waits for this grid before reading units
+    const int gid = blockIdx.x * blockDim.x + threadIdx.x;
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < a.header_words; i += blockDim.x) a.header[i] = 0u;
+    if (gid < a.n_q) {
+        const int b = find_seq(a.q_off, a.n_seqs, gid);
+        a.rows[gid] = RowDesc{gid, b, eligible_count(a.q_pos[gid], a.k_off[b + 1] - a.k_off[b]), 0};
+    }
+    if (gid < a.n_units) {
+        const int tau = gid / a.splits, s = gid % a.splits;
+        int lo = 0, hi = a.n_seqs - 1;   // the sequence whose tiles hold tile tau
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (a.tile_base[mid] <= tau) lo = mid; else hi = mid - 1;
+        }
+        const int b = lo;
+        const int q0 = a.q_off[b], nq = a.q_off[b + 1] - q0;
+        const int ntile = a.tile_base[b + 1] - a.tile_base[b];
+        const int jj = ntile - 1 - (tau - a.tile_base[b]);   // longest causal tiles first
+        const int r0 = q0 + jj * a.TQ;
+        const int nr = min(a.TQ, nq - jj * a.TQ);
+        const int L = a.k_off[b + 1] - a.k_off[b];
+        int maxnc = 0;
+        for (int r = r0; r < r0 + nr; ++r) maxnc = max(maxnc, eligible_count(a.q_pos[r], L));
+        const int nkt = (maxnc + 127) / 128;
+        a.units[gid] = TcUnit{r0, nr, nkt * s / a.splits, nkt * (s + 1) / a.splits, r0, a.k_off[b], {0, 0}};
+    }
+}
+
 // Rows [r0, r0 + n) of a row array, with their query rows made relative to r0 (a row chunk whose
 // queries sit in a buffer of their own).
 __global__ void chunk_rows_kernel(const RowDesc* rows, int32_t r0, int32_t n, RowDesc* out)

@@ -142,3 +142,26 @@ def test_pivot_and_hisa_argument_errors():
     for k, B, keep in ((4, 100, 4), (4, 128, 0), (0, 128, 4)):
         assert lib.hisa_index(lay.ref(), P(0x1000), P(0x2000), P(0x3000), P(0x5000), k, B, keep, P(0x4000), None,
                               P(0x10000), ctypes.c_size_t(1 << 30), None) == 2
+
+
+def test_layer_schedule_host_function_matches_oracle():
+    """dsa_index_layers_source (host-only) against the oracle's stepwise reading of IndexCache and MLI."""
+    import oracle
+    for n in range(1, 12):
+        for r in (1, 2, 3, 4, 8):
+            for lag in (0, 1):
+                want = oracle.layer_sources(n, r, lag)
+                got = [dsa.index_layers_source(l, r, lag) for l in range(n)]
+                assert got == want, (n, r, lag)
+    assert dsa.index_layers_source(-1, 2, 0) == -1
+    assert dsa.index_layers_source(3, 0, 0) == -1
+    assert dsa.index_layers_source(3, 2, 2) == -1
+
+
+def test_checked_build_exports_the_same_entry_points():
+    """libdsaidx_checked.so (the build whose kernels verify their device-side indices) exports every
+    declared entry point too."""
+    path = os.path.join(ROOT, "sparse_attention_indexer_04_b200", "libdsaidx_checked.so")
+    lib = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(lib, name), name

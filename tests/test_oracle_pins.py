@@ -416,3 +416,26 @@ def test_pair_scores_address_the_query_sequence_keys():
     seq_of_row = [0, 0, 1, 1, 1, 2, 2, 2]
     got = oracle.pair_scores(bt, rows, keys)
     assert got.tolist() == [(seq_of_row[r] + 1.0) * d for r in rows]
+
+
+# ------------------------------------------------------ cross-layer reuse
+
+LAYERS = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "layer_schedules.json")))
+
+
+@pytest.mark.parametrize("case", LAYERS["cases"], ids=lambda c: f"n{c['n_layers']}_r{c['retain_every']}_lag{c['lag']}")
+def test_layer_sources_match_hand_schedules(case):
+    assert oracle.layer_sources(case["n_layers"], case["retain_every"], case["lag"]) == case["sources"]
+
+
+def test_layer_topk_is_each_source_layers_dense_topk():
+    """The selections are the dense oracle's top-k of the source layer's own inputs; with one full
+    layer in every layer and no lag, every layer keeps its own."""
+    bs = [workloads.tiny_integer(seed=60 + l, T=40, H=2, d=32, k=6) for l in range(4)]
+    own = [oracle.dense(b, k=6)["idx"] for b in bs]
+    sel = oracle.layer_topk(bs, 6, 1, 0)
+    assert all(np.array_equal(a, b) for a, b in zip(sel, own))
+    sel = oracle.layer_topk(bs, 6, 2, 1)           # sources [0, 0, 0, 2]
+    for got, s in zip(sel, [0, 0, 0, 2]):
+        assert np.array_equal(got, own[s])
+    assert not np.array_equal(own[0], own[2])     # the layers' inputs differ, so the sources matter
