@@ -221,9 +221,9 @@ dsa_status launch_score(const RowDesc* rows, int32_t n_rows, int32_t max_cols, c
     const dim3 grid(n_rows, (cols + kSimtCols - 1) / kSimtCols);
     const size_t smem = size_t(H) * D * sizeof(float) + size_t(H) * sizeof(float);
     switch (D) {
-    case 32: DSA_LAUNCH(kProfScoreSimt, st, score_simt_kernel<32, KT><<<grid, kSimtCols, smem, st>>>(a)); break;
-    case 64: DSA_LAUNCH(kProfScoreSimt, st, score_simt_kernel<64, KT><<<grid, kSimtCols, smem, st>>>(a)); break;
-    default: DSA_LAUNCH(kProfScoreSimt, st, score_simt_kernel<128, KT><<<grid, kSimtCols, smem, st>>>(a)); break;
+    case 32: DSA_LAUNCH(kProfScoreSimt, st, score_simt_kernel<32, KT><<<grid, kSimtThreads, smem, st>>>(a)); break;
+    case 64: DSA_LAUNCH(kProfScoreSimt, st, score_simt_kernel<64, KT><<<grid, kSimtThreads, smem, st>>>(a)); break;
+    default: DSA_LAUNCH(kProfScoreSimt, st, score_simt_kernel<128, KT><<<grid, kSimtThreads, smem, st>>>(a)); break;
     }
     return launched();
 }
@@ -1313,24 +1313,22 @@ dsa_status hisa_index(const dsa_batch* b, const void* Q, const void* K, const fl
     if ((s = check_ws(ws, ws_bytes, hisa_plan(nullptr, b, hi, k, B, keep, &p))) != DSA_OK) return s;
     hisa_plan(static_cast<char*>(ws), b, hi, k, B, keep, &p);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if ((s = clear_status(ws, st)) != DSA_OK) return s;
     const int32_t nq = b->num_queries;
-    if (nq == 0) return DSA_OK;
+    if (nq == 0) return clear_status(ws, st);
+    g_status = static_cast<uint32_t*>(ws);   // hisa_setup_kernel clears the header
     const int H = b->num_heads, D = b->head_dim;
     int32_t* kept = kept_out ? kept_out : p.kept;
     const unsigned g = (nq + 255) / 256;
 
     DSA_LAUNCH(kProfSetup, st, hisa_setup_kernel<<<(nq + 256) / 256, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos,
-                                                    b->num_seqs, nq, B, p.block_base, p.block_rows, p.query_off));
+                                                    b->num_seqs, nq, B, p.block_base, p.block_rows, p.query_off,
+                                                    static_cast<uint32_t*>(ws), (int32_t)(kHeaderBytes / 4)));
     if ((s = launched()) != DSA_OK) return s;
     // Coarse stage: middle blocks scored on their pooled keys, top `keep` kept.
     const int32_t max_mid = std::max(0, (hi.max_k + B - 1) / B - 2);
     s = score_and_select<float>(p.block_rows, nq, max_mid, identity_map(1), Q, W, H, D, pooled, p.block_base, p.S,
                                 keep, p.mid, keep, nullptr, st);
     if (s != DSA_OK) return s;
-    DSA_LAUNCH(kProfSetup, st, hisa_kept_kernel<<<g, 256, 0, st>>>(p.block_rows, p.mid, keep, b->q_pos, b->k_offsets, nq, B, kept,
-                                        p.token_rows));
-    if ((s = launched()) != DSA_OK) return s;
     // Fine stage: the indexer over the tokens of the kept blocks.
     ColMap m{};
     m.kind = kMapBlocks;
@@ -1339,7 +1337,24 @@ dsa_status hisa_index(const dsa_batch* b, const void* Q, const void* K, const fl
     m.list_ld = keep + 2;
     const std::vector<int32_t> qoff = iota_host(nq);
     const TcSource src{Q, nq, W, p.query_off, qoff.data(), nq};
-    return tc_score_and_select(p.token_rows, nq, src, H, D, K, b->num_keys, b->k_offsets, m, (keep + 2) * B, p.S,
+    const int32_t tok_cols = (keep + 2) * B;
+    const int64_t ld_tok = score_ld(tok_cols);
+    if (chunk_rows(nq, ld_tok) >= nq) {
+        // one scoring launch: kept blocks, token rows and its units in one kernel (a warp per query)
+        const int32_t splits = tc_splits(tc_count_tiles(qoff.data(), nq, 0, nq, tc_tile_rows(H)), tok_cols);
+        DSA_LAUNCH(kProfSetup, st, launch_pdl(latency_bound(nq), hisa_kept_units_kernel, (nq + 7) / 8, 256, 0, st,
+                                              p.block_rows, p.mid, keep, b->q_pos, b->k_offsets, nq, B, splits, kept,
+                                              p.token_rows, p.units));
+        if ((s = launched()) != DSA_OK) return s;
+        s = tc_score(p.token_rows, nq, 0, src, H, D, K, b->num_keys, b->k_offsets, m, tok_cols, p.S, ld_tok, p.units,
+                     p.tile_base, static_cast<uint32_t*>(ws), st, true);
+        if (s != DSA_OK) return s;
+        return launch_select(p.token_rows, nq, tok_cols, k, m, p.S, ld_tok, false, idx, k, nullptr, 0, st, p.split);
+    }
+    DSA_LAUNCH(kProfSetup, st, hisa_kept_kernel<<<g, 256, 0, st>>>(p.block_rows, p.mid, keep, b->q_pos, b->k_offsets, nq, B, kept,
+                                        p.token_rows));
+    if ((s = launched()) != DSA_OK) return s;
+    return tc_score_and_select(p.token_rows, nq, src, H, D, K, b->num_keys, b->k_offsets, m, tok_cols, p.S,
                                p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k, nullptr, st, p.split);
 }
 

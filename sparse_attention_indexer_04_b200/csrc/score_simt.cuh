@@ -1,18 +1,26 @@
 // CUDA-core scoring of rows against (mapped) key columns, fp32 FMA.
 //
 // Used where the operand is not a bf16 tensor-core tile: HISA's pooled fp32
-// block keys, and small or irregular rows.  One CTA scores one row against
-// 128 consecutive columns; thread c holds its key in registers and walks
-// the row's H heads, I = sum_h w_h * max(0, q_h . k), each dot product
-// accumulated in fp32 as four interleaved partial sums (four independent
-// FMA chains instead of one 128-long chain).
+// block keys.  A CTA scores one row against kSimtCols consecutive columns,
+// four lanes (a quad) per two columns: lane j of the quad holds the
+// 4-dimension groups j, j+4, j+8, ... of both columns' keys in registers (so
+// a quad's loads of q_h read 64 consecutive bytes, and each feeds both
+// columns), computes the partial dot products of every head over them, and
+// two xor shuffles give every lane of the quad the head's full q_h . k; then
+// I = sum_h w_h * max(0, q_h . k), in fp32.  Splitting the dimensions (not
+// the heads) keeps one read of each key and a quarter of its registers per
+// lane, so an SM holds enough warps to hide the FMA and shared-memory
+// latencies of this short, latency-bound launch; the shared-memory reads of
+// q are its limit, hence two columns per quad.
 #pragma once
 
 #include "common.cuh"
 
 namespace dsa {
 
-constexpr int kSimtCols = 128;
+constexpr int kSimtColsPerQuad = 2;           // columns per quad: each q load feeds both
+constexpr int kSimtThreads = 256;
+constexpr int kSimtCols = kSimtThreads / 4 * kSimtColsPerQuad;   // columns per CTA
 
 struct ScoreArgs {
     const RowDesc* rows;
@@ -29,36 +37,38 @@ struct ScoreArgs {
     int32_t pad_;
 };
 
+// The 4-dimension groups part, part + 4, part + 8, ... of a key row of D elements (bf16 or fp32) into
+// registers: D / 4 values.
 template <int D>
-__device__ __forceinline__ void load_key(const __nv_bfloat16* kp, float* kr)
+__device__ __forceinline__ void load_key_part(const __nv_bfloat16* kp, int part, float* kr)
 {
-    const uint4* p = reinterpret_cast<const uint4*>(kp);
+    const uint2* p = reinterpret_cast<const uint2*>(kp);   // 4 bf16 per 8 bytes
 #pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-        const uint4 v = __ldg(p + j);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            kr[8 * j + 2 * e] = __uint_as_float(w[e] << 16);
-            kr[8 * j + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-        }
+    for (int m = 0; m < D / 16; ++m) {
+        const uint2 v = __ldg(p + 4 * m + part);
+        kr[4 * m] = __uint_as_float(v.x << 16);
+        kr[4 * m + 1] = __uint_as_float(v.x & 0xffff0000u);
+        kr[4 * m + 2] = __uint_as_float(v.y << 16);
+        kr[4 * m + 3] = __uint_as_float(v.y & 0xffff0000u);
     }
 }
 
 template <int D>
-__device__ __forceinline__ void load_key(const float* kp, float* kr)
+__device__ __forceinline__ void load_key_part(const float* kp, int part, float* kr)
 {
     const float4* p = reinterpret_cast<const float4*>(kp);
 #pragma unroll
-    for (int j = 0; j < D / 4; ++j) {
-        const float4 v = __ldg(p + j);
-        kr[4 * j] = v.x; kr[4 * j + 1] = v.y; kr[4 * j + 2] = v.z; kr[4 * j + 3] = v.w;
+    for (int m = 0; m < D / 16; ++m) {
+        const float4 v = __ldg(p + 4 * m + part);
+        kr[4 * m] = v.x; kr[4 * m + 1] = v.y; kr[4 * m + 2] = v.z; kr[4 * m + 3] = v.w;
     }
 }
 
 template <int D, typename KT>
-__global__ void __launch_bounds__(kSimtCols) score_simt_kernel(ScoreArgs a)
+__global__ void __launch_bounds__(kSimtThreads) score_simt_kernel(ScoreArgs a)
 {
+    constexpr int DQ = D / 4;   // dimensions per lane
+    static_assert(D % 16 == 0, "4-dimension groups, four per quad");
     extern __shared__ float sm[];
     const int r = blockIdx.x;
     const RowDesc rd = a.rows[r];
@@ -67,35 +77,76 @@ __global__ void __launch_bounds__(kSimtCols) score_simt_kernel(ScoreArgs a)
     if (col0 >= lim) return;
     float* sq = sm;
     float* sw = sm + a.H * D;
-    const __nv_bfloat16* q = a.Q + (int64_t)rd.qrow * a.H * D;
-    for (int i = threadIdx.x; i < a.H * D; i += kSimtCols) sq[i] = __bfloat162float(q[i]);
-    for (int h = threadIdx.x; h < a.H; h += kSimtCols) sw[h] = a.W[(int64_t)rd.qrow * a.H + h];
-    __syncthreads();
-    const int col = col0 + threadIdx.x;
-    float out = -INFINITY;
-    if (col < rd.ncols) {
-        const int32_t key = map_col(a.map, rd, col);
-        const KT* kp = reinterpret_cast<const KT*>(a.K) + (int64_t)(a.k_base[rd.seq] + key) * D;
-        float kr[D];
-        load_key<D>(kp, kr);
-        float acc = 0.f;
-#pragma unroll 2
-        for (int h = 0; h < a.H; ++h) {
-            const float4* qh = reinterpret_cast<const float4*>(sq + h * D);
-            float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+    // the row's query (H x D bf16, 16-byte loads, all of a thread's in flight at once) and weights
+    const uint4* q = reinterpret_cast<const uint4*>(a.Q + (int64_t)rd.qrow * a.H * D);
+    const int n8 = a.H * D / 8;
+    constexpr int kPer = 64 * 128 / 8 / kSimtThreads;   // loads per thread for the largest query
 #pragma unroll
-            for (int i = 0; i < D / 4; ++i) {
-                const float4 qv = qh[i];
-                d0 = fmaf(qv.x, kr[4 * i], d0);
-                d1 = fmaf(qv.y, kr[4 * i + 1], d1);
-                d2 = fmaf(qv.z, kr[4 * i + 2], d2);
-                d3 = fmaf(qv.w, kr[4 * i + 3], d3);
+    for (int u = 0; u < kPer; ++u) {
+        const int i = threadIdx.x + u * kSimtThreads;
+        if (i < n8) {
+            const uint4 v = __ldg(q + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                sq[8 * i + 2 * e] = __uint_as_float(w[e] << 16);
+                sq[8 * i + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
             }
-            acc = fmaf(sw[h], fmaxf((d0 + d1) + (d2 + d3), 0.f), acc);
         }
-        out = acc + 0.f;   // -0 -> +0
     }
-    if (col < lim) a.S[(int64_t)r * a.ld_s + col] = out;
+    for (int h = threadIdx.x; h < a.H; h += kSimtThreads) sw[h] = a.W[(int64_t)rd.qrow * a.H + h];
+    __syncthreads();
+    const int part = threadIdx.x & 3;   // which 4-dimension groups
+    constexpr int C = kSimtColsPerQuad;
+    const int colq = col0 + (threadIdx.x >> 2) * C;   // the quad's first column
+    float kr[C][DQ];
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        if (colq + c < rd.ncols) {
+            const int32_t key = map_col(a.map, rd, colq + c);
+            const KT* kp = reinterpret_cast<const KT*>(a.K) + (int64_t)(a.k_base[rd.seq] + key) * D;
+            load_key_part<D>(kp, part, kr[c]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < DQ; ++i) kr[c][i] = 0.f;
+        }
+    }
+    float acc[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) acc[c] = 0.f;
+#pragma unroll 2
+    for (int h = 0; h < a.H; ++h) {
+        const float4* qh = reinterpret_cast<const float4*>(sq + h * D) + part;
+        float d0[C], d1[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) { d0[c] = 0.f; d1[c] = 0.f; }
+#pragma unroll
+        for (int i = 0; i < DQ / 4; ++i) {
+            const float4 qv = qh[4 * i];   // dimensions 4 (4 i + part) .. +3
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                d0[c] = fmaf(qv.x, kr[c][4 * i], d0[c]);
+                d1[c] = fmaf(qv.y, kr[c][4 * i + 1], d1[c]);
+                d0[c] = fmaf(qv.z, kr[c][4 * i + 2], d0[c]);
+                d1[c] = fmaf(qv.w, kr[c][4 * i + 3], d1[c]);
+            }
+        }
+        const float w = sw[h];
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            float dot = d0[c] + d1[c];
+            dot += __shfl_xor_sync(0xffffffffu, dot, 1);   // the quad's four parts
+            dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+            acc[c] = fmaf(w, fmaxf(dot, 0.f), acc[c]);
+        }
+    }
+    if (part < C) {   // lane c of the quad writes column c
+        float v = acc[0];
+#pragma unroll
+        for (int c = 1; c < C; ++c) v = part == c ? acc[c] : v;
+        const int col = colq + part;
+        if (col < lim) a.S[(int64_t)r * a.ld_s + col] = col < rd.ncols ? v + 0.f : -INFINITY;   // -0 -> +0
+    }
 }
 
 }  // namespace dsa

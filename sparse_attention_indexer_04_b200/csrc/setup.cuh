@@ -270,10 +270,14 @@ __global__ void hisa_pool_kernel(const __nv_bfloat16* K, const int32_t* k_off, i
 // HISA set-up in one launch: every CTA writes the block-scoring rows (the
 // middle blocks 1 .. last-1 of query t; column c is block c + 1) and the
 // per-query segment offsets query_off[t] = t of its queries; CTA 0 also
-// writes block_base (first pooled block of each sequence).
+// writes block_base (first pooled block of each sequence) and clears the
+// workspace header.
 __global__ void hisa_setup_kernel(const int32_t* q_off, const int32_t* k_off, const int32_t* q_pos, int32_t n_seqs,
-                                  int32_t n_q, int32_t B, int32_t* block_base, RowDesc* rows, int32_t* query_off)
+                                  int32_t n_q, int32_t B, int32_t* block_base, RowDesc* rows, int32_t* query_off,
+                                  uint32_t* header, int32_t header_words)
 {
+    if (blockIdx.x == 0)   // the workspace header (status word, select counters) starts the call at zero
+        for (int i = threadIdx.x; i < header_words; i += blockDim.x) header[i] = 0u;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         int32_t acc = 0;
         for (int b = 0; b < n_seqs; ++b) {
@@ -318,6 +322,44 @@ __global__ void hisa_kept_kernel(const RowDesc* block_rows, const int32_t* mid, 
     }
     for (int j = m; j < keep + 2; ++j) out[j] = -1;
     token_rows[t] = RowDesc{t, br.seq, ncols, t};
+}
+
+// Kept blocks and token rows (as hisa_kept_kernel) and the token-scoring work units, one warp per
+// query: the lanes read the query's selected middle blocks together (ascending, then -1), and the
+// query's `splits` units cover the kept blocks' key tiles (a query is a segment of one row).
+__global__ void hisa_kept_units_kernel(const RowDesc* block_rows, const int32_t* mid, int32_t keep,
+                                       const int32_t* q_pos, const int32_t* k_off, int32_t n_q, int32_t B,
+                                       int32_t splits, int32_t* kept, RowDesc* token_rows, TcUnit* units)
+{
+    grid_dep_wait();     // the block selection comes from the previous kernel
+    grid_dep_launch();
+    const int t = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+    if (t >= n_q) return;   // (uniform per warp)
+    const RowDesc br = block_rows[t];
+    const int L = k_off[br.seq + 1] - k_off[br.seq];
+    const int n = eligible_count(q_pos[t], L);
+    const int last = n > 0 ? (n - 1) / B : 0;
+    int32_t* out = kept + (int64_t)t * (keep + 2);
+    // the selected middle blocks are packed first: count them a warp's width at a time
+    int n_mid = 0;
+    for (int j0 = 0; j0 < keep; j0 += 32) {
+        const int j = j0 + lane;
+        const int32_t v = j < keep ? mid[(int64_t)t * keep + j] : -1;
+        if (v >= 0 && n > 0) out[1 + j] = v;
+        n_mid += __popc(__ballot_sync(0xffffffffu, v >= 0));
+    }
+    if (n == 0) n_mid = 0;
+    const int m = n > 0 ? 1 + n_mid + (last > 0 ? 1 : 0) : 0;   // kept blocks
+    if (lane == 0 && n > 0) {
+        out[0] = 0;
+        if (last > 0) out[1 + n_mid] = last;
+    }
+    for (int j = m + lane; j < keep + 2; j += 32) out[j] = -1;
+    const int ncols = m > 0 ? (m - 1) * B + (n - last * B) : 0;
+    if (lane == 0) token_rows[t] = RowDesc{t, br.seq, ncols, t};
+    const int nkt = (ncols + 127) / 128;
+    for (int s = lane; s < splits; s += 32)
+        units[(int64_t)t * splits + s] = TcUnit{t, 1, nkt * s / splits, nkt * (s + 1) / splits, t, k_off[br.seq], {0, 0}};
 }
 
 // ------------------------------------------------------ tensor-core units
