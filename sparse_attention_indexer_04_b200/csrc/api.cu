@@ -229,10 +229,14 @@ dsa_status launch_score(const RowDesc* rows, int32_t n_rows, int32_t max_cols, c
 }
 
 // Threads per row of the streaming select: 256 when rows fill the GPU several times over, 512
-// when there are few rows or k is large (each row's phases are latency-bound).  Measured on the
-// 32K prefill (32768 rows: 256 best), the 16 x 32K decode (32 rows: 512 best) and PIVOT's top-8192
-// candidate selection (512 best).
-int select_threads(int32_t n_rows, int32_t k) { return n_rows < 2 * 148 || k >= 4096 ? 512 : 256; }
+// when there are few rows or k is large (each row's phases are latency-bound), 1024 for k of 8192
+// or more (the candidate buffer then takes most of the shared memory: one CTA per SM).  Measured on
+// the 32K prefill (32768 rows: 256 best), the 16 x 32K decode (32 rows: 512 best) and PIVOT's
+// top-8192 candidate selection at 128K (1024: 3.12 ms against 3.44 with 512).
+int select_threads(int32_t n_rows, int32_t k)
+{
+    return k >= 8192 ? 1024 : n_rows < 2 * 148 || k >= 4096 ? 512 : 256;
+}
 
 // Dynamic shared memory the select kernels may take: a CTA's 227 KB less their static shared
 // memory (SelScalars: the radix histogram and scalars, about 1.2 KB; 4 KB reserved).
@@ -321,6 +325,10 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
         return launched();
     }
     switch (select_threads(n_rows, k)) {
+    case 1024:
+        if ((s = set_smem(select_stream_kernel<1024>, smem)) != DSA_OK) return s;
+        DSA_LAUNCH(kProfSelect, st, launch_pdl(latency_bound(n_rows), select_stream_kernel<1024>, n_rows, 1024, smem, st, a));
+        break;
     case 512:
         if ((s = set_smem(select_stream_kernel<512>, smem)) != DSA_OK) return s;
         DSA_LAUNCH(kProfSelect, st, launch_pdl(latency_bound(n_rows), select_stream_kernel<512>, n_rows, 512, smem, st, a));

@@ -2,10 +2,8 @@
 // cluster (2 <= P <= 8) and share the steps of select.cuh through distributed shared memory,
 // instead of handing candidates to one finishing CTA through L2.
 //
-//   1. threshold: the row's sample (the same m/32 runs of 32 columns select_stream_kernel reads)
-//      is split among the P CTAs by runs; each counts its part into its own histogram and the
-//      leader (cluster rank 0) sums the P histograms digit by digit, so tau is the key one CTA
-//      would find over the whole sample;
+//   1. threshold: every CTA ranks the row's whole sample (the same m/32 runs of 32 columns
+//      select_stream_kernel reads) by itself, the same way, so all find the same tau;
 //   2. each CTA appends the columns of its chunk with key >= tau to its own candidate buffer;
 //   3. the CTAs copy their candidates into the leader's buffer (offsets from one atomic on the
 //      leader's counter); if the union holds >= k entries and nothing overflowed, the leader
@@ -29,11 +27,8 @@ constexpr int kClusterMaxParts = 8;
 
 // Scalars the row's CTAs exchange; the leader's copy is the one read.
 struct alignas(16) ClusterShared {
-    uint32_t lo[kClusterMaxParts];   // each CTA's sample key range
-    uint32_t hi[kClusterMaxParts];
     uint32_t gt[kClusterMaxParts];   // each CTA's marked counts (> T, == T)
     uint32_t eq[kClusterMaxParts];
-    uint32_t step[3];                // the current radix digit: digit, keys above it, whole-digit flag
     uint32_t count;                  // candidates in the leader's buffer
     uint32_t overflow;               // nonzero: some buffer overflowed
     uint32_t T;                      // the row's k-th key
@@ -46,74 +41,6 @@ struct alignas(16) ClusterShared {
 __host__ __device__ inline size_t cluster_smem_bytes(size_t sample_bytes, int cap, int chunk_words)
 {
     return sample_bytes + (size_t)cap * 16 + (size_t)chunk_words * 8;
-}
-
-// radix_select over keys spread over the cluster's CTAs (count of them in this CTA, given by
-// get): each pass counts into the CTA's own histogram, the leader's warp 0 sums the P
-// histograms and picks the digit.  lo, hi and krem are the same in every CTA.  Two cluster
-// barriers per pass.
-template <int NT, typename Get>
-__device__ __forceinline__ uint32_t cluster_radix(cg::cluster_group& cl, ClusterShared* lead, int P, Get get,
-                                                  int count, int& krem, uint32_t lo, uint32_t hi, int stop_bits,
-                                                  SelScalars<NT>& sh)
-{
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    int top = 32 - __clz(hi - lo);
-    const int stop = stop_bits > 0 ? max(top - stop_bits, 0) : 0;
-    uint32_t prefix = 0;
-    while (top > stop) {
-        const int shift = max(top - 8, 0), width = top - shift;
-        __syncthreads();
-        for (int i = tid; i < 256; i += NT) sh.hist[i] = 0;
-        __syncthreads();
-        for (int i = tid; i < count; i += NT) {
-            const uint32_t rel = get(i) - lo;
-            if (((rel >> 1) >> (top - 1)) == prefix) atomicAdd(&sh.hist[(rel >> shift) & ((1u << width) - 1u)], 1u);
-        }
-        cl.sync();   // every CTA's histogram is complete
-        if (cl.block_rank() == 0 && warp == 0) {
-            uint32_t c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            for (int q = 0; q < P; ++q) {
-                const uint32_t* hq = cl.map_shared_rank(sh.hist, q);
-#pragma unroll
-                for (int b = 0; b < 8; ++b) c[b] += hq[8 * lane + b];
-            }
-            uint32_t tot = 0;
-#pragma unroll
-            for (int b = 0; b < 8; ++b) tot += c[b];
-            uint32_t incl = tot;   // keys in the digits of lanes >= this lane
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t x = __shfl_down_sync(0xffffffffu, incl, o);
-                if (lane + o < 32) incl += x;
-            }
-            const uint32_t above = incl - tot;
-            if (above < (uint32_t)krem && (uint32_t)krem <= incl) {
-                uint32_t acc = above;
-                int b = 7;
-                for (; b > 0; --b) {
-                    if (acc + c[b] >= (uint32_t)krem) break;
-                    acc += c[b];
-                }
-                lead->step[0] = 8 * lane + b;
-                lead->step[1] = acc;
-                lead->step[2] = acc + c[b] == (uint32_t)krem;   // the whole digit is taken
-            }
-        }
-        cl.sync();   // the digit is known
-        prefix = (prefix << width) | lead->step[0];
-        krem -= (int)lead->step[1];
-        const bool whole = lead->step[2] != 0;
-        top = shift;
-        if (stop_bits == 0 && top > 0 && whole) {
-            const uint32_t edge = lo + (prefix << top);
-            if (edge > 0) {
-                krem = 0;
-                return edge - 1;
-            }
-        }
-    }
-    return lo + (prefix << top);
 }
 
 // Grid: P CTAs per row (blockIdx.x = row * P + cluster rank), launched as clusters of P.
@@ -156,39 +83,11 @@ __global__ void __launch_bounds__(NT, 1) select_cluster_kernel(SelectArgs a, int
     }
     cl.sync();   // the leader's counters are zero before any CTA adds to them
 
-    // ---- 1. tau from the row's sample, split among the CTAs by runs
+    // ---- 1. tau: every CTA ranks the whole sample itself, the same way, so every CTA holds the same
+    // tau with no cluster exchange (measured: the sample split among the CTAs, its digits summed in the
+    // leader across two cluster barriers each, was 2-3.5 us slower per row)
     uint32_t tau = 0;
-    if (n > k && n > cap) {
-        const int m = select_sample_size(n, k);
-        const uint32_t R = (uint32_t)(m / 32);
-        const uint32_t ra = R * (uint32_t)p / (uint32_t)P, rb = R * (uint32_t)(p + 1) / (uint32_t)P;
-        const int mine = (int)(rb - ra) * 32;
-        uint32_t lo = 0xffffffffu, hi = 0u;
-        for (int e = tid; e < mine; e += NT) {
-            const uint32_t run = ra + (uint32_t)(e >> 5);   // r n < 2^31
-            const int col = (int)(((run * (uint32_t)n) / R) & ~31u) + (e & 31);
-            const uint32_t u = score_key(__ldg(src + min(col, n - 1)));
-            sample[e] = u;
-            lo = min(lo, u);
-            hi = max(hi, u);
-        }
-        block_key_range<NT>(lo, hi, sh.scratch);   // also publishes the sample to the CTA
-        if (tid == 0) {
-            lead->lo[p] = lo;
-            lead->hi[p] = hi;
-        }
-        cl.sync();   // every CTA's range is in the leader
-        lo = 0xffffffffu;
-        hi = 0u;
-        for (int q = 0; q < P; ++q) {
-            lo = min(lo, lead->lo[q]);
-            hi = max(hi, lead->hi[q]);
-        }
-        const float expect = (float)k * m / n;
-        int rank = (int)ceilf(expect + 4.f * sqrtf(expect) + 4.f);
-        rank = min(rank, m);
-        tau = cluster_radix<NT>(cl, lead, P, [&](int i) { return sample[i]; }, mine, rank, lo, hi, 16, sh);
-    }
+    if (n > k) tau = sel_threshold<NT>(src, n, k, cap, sample, sh);
 
     // ---- 2. this chunk's candidates; 3. into the leader's buffer
     if (n > k) sel_append<NT>(src, c0, c1, tau, cand, cap, sh);
