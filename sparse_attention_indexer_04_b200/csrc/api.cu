@@ -24,10 +24,11 @@ namespace {
 
 constexpr int32_t kMaxK = 16384;
 constexpr int32_t kMaxCand = 16384;
-// Bytes of materialised score rows per launch: 1 GiB keeps a 32K prefill's scoring launches at
-// ~1000 units (about 7 waves of 148 SMs), where 256 MiB (256 units, 1.7 waves) lost ~14 % to
-// the last wave.
-constexpr size_t kScoreBudget = size_t(1024) << 20;
+// Bytes of materialised score rows per launch: 4 GiB holds a whole 32K prefill (one scoring launch
+// of 4096 units and one select, through dense_topk_one_launch).  Measured on that prefill: 7.33 ms
+// per step against 7.40 (2 GiB, two chunks) and 7.37-7.42 (1 GiB, four); 256 MiB (256 units, 1.7
+// waves per launch) lost ~14 % to the last wave.
+constexpr size_t kScoreBudget = size_t(4096) << 20;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -581,14 +582,16 @@ struct DensePlan {
     SelectSplit split;
 };
 
-// k = 0: the scores-only entry point (no score buffer, no select).
-size_t dense_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, DensePlan* p)
+// k = 0: the scores-only entry point (no score buffer, no select).  max_chunk: the caller scores
+// at most this many rows at a time (the score buffer is sized for it).
+size_t dense_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, DensePlan* p,
+                  int32_t max_chunk = INT32_MAX)
 {
     Carver c{base};
     const int32_t nq = std::max(1, b->num_queries);
     p->rows = c.take<RowDesc>(nq);
     const int64_t ld = score_ld(hi.max_k);
-    const int32_t chunk = k == 0 ? nq : chunk_rows(nq, ld);
+    const int32_t chunk = k == 0 ? nq : std::min(max_chunk, chunk_rows(nq, ld));
     const TcSource src{nullptr, 0, nullptr, nullptr, b->q_offsets_host, b->num_seqs};
     p->units = c.take<TcUnit>(tc_unit_capacity(src, b->num_queries, chunk, b->num_heads, hi.max_k));
     p->tile_base = c.take<int32_t>(b->num_seqs + 1);
@@ -631,7 +634,8 @@ int32_t host_chunk_rows(int32_t nq, int64_t ld)
 
 size_t host_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, DensePlan* dp, HostPlan* p)
 {
-    const size_t inner = dense_plan(base, b, hi, k, dp);
+    const size_t inner = dense_plan(base, b, hi, k, dp,
+                                    host_chunk_rows(std::max(1, b->num_queries), score_ld(hi.max_k)));
     Carver c{base};
     c.off = align256(inner);
     const int32_t nq = std::max(1, b->num_queries);
