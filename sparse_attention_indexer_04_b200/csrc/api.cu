@@ -15,6 +15,7 @@
 #include "score_tc.cuh"
 #include "select.cuh"
 #include "select_cluster.cuh"
+#include "select_regs.cuh"
 #include "reuse.cuh"
 #include "setup.cuh"
 
@@ -412,17 +413,18 @@ int32_t tc_count_tiles(const int32_t* off, int n_seqs, int64_t row_base, int64_t
     return (int32_t)n;
 }
 
-// Key-range splits per query tile when there are fewer tiles than SMs (decode).
-int32_t tc_splits(int32_t tiles, int32_t max_cols)
+// Key-range splits per query tile when there are fewer tiles than SMs (decode).  Units keep at
+// least min_tiles key tiles (8 for the dense scan; HISA's short rows use 1 and 2).
+int32_t tc_splits(int32_t tiles, int32_t max_cols, int32_t min_tiles = 8)
 {
     const int32_t kt = (max_cols + 127) / 128;
-    if (tiles <= 0 || tiles >= 148 || kt < 16) return 1;
+    if (tiles <= 0 || tiles >= 148 || kt < 2 * min_tiles) return 1;
     // One CTA fills an SM, so the units run in waves of 148: pick the split count s (units of at
-    // least 8 key tiles) minimising waves(s) * (ceil(kt / s) + 2), the 2 standing for a CTA's
-    // start-up (barriers, TMEM, the query tile) in key tiles.
+    // least min_tiles key tiles) minimising waves(s) * (ceil(kt / s) + 2), the 2 standing for a
+    // CTA's start-up (barriers, TMEM, the query tile) in key tiles.
     int32_t best = 1;
     int64_t best_cost = INT64_MAX;
-    for (int32_t s = 1; s <= kt / 8; ++s) {
+    for (int32_t s = 1; s <= kt / min_tiles; ++s) {
         const int64_t waves = (int64_t(tiles) * s + 147) / 148;
         const int64_t cost = waves * ((kt + s - 1) / s + 2);
         if (cost < best_cost) { best_cost = cost; best = s; }
@@ -470,12 +472,16 @@ dsa_status launch_tc_shape(const CUtensorMap& mq, const CUtensorMap& mk, const C
     const int smem = std::max((int)SH::smem_bytes(n_acc, stages), 120 * 1024);
     dsa_status s;
     if (a.gather) {
-        if ((s = set_smem(score_tc_kernel<D, H, true>, smem)) != DSA_OK) return s;
-        DSA_LAUNCH(kProfScoreTc, st, launch_pdl(latency_bound(n_units), score_tc_kernel<D, H, true>, n_units,
+        if ((s = set_smem(score_tc_kernel<D, H, kTcGather>, smem)) != DSA_OK) return s;
+        DSA_LAUNCH(kProfScoreTc, st, launch_pdl(latency_bound(n_units), score_tc_kernel<D, H, kTcGather>, n_units,
                                                 kTcThreads, smem, st, mq, mk, mkg, args));
+    } else if (a.planes > 1 || a.block_tiles) {
+        if ((s = set_smem(score_tc_kernel<D, H, kTcBlocks>, smem)) != DSA_OK) return s;
+        DSA_LAUNCH(kProfScoreTc, st, launch_pdl(latency_bound(n_units), score_tc_kernel<D, H, kTcBlocks>, n_units,
+                                                kTcThreadsTiles, smem, st, mq, mk, mkg, args));
     } else {
-        if ((s = set_smem(score_tc_kernel<D, H, false>, smem)) != DSA_OK) return s;
-        DSA_LAUNCH(kProfScoreTc, st, launch_pdl(latency_bound(n_units), score_tc_kernel<D, H, false>, n_units,
+        if ((s = set_smem(score_tc_kernel<D, H, kTcTiles>, smem)) != DSA_OK) return s;
+        DSA_LAUNCH(kProfScoreTc, st, launch_pdl(latency_bound(n_units), score_tc_kernel<D, H, kTcTiles>, n_units,
                                                 kTcThreadsTiles, smem, st, mq, mk, mkg, args));
     }
     return launched();
@@ -496,20 +502,33 @@ dsa_status launch_tc_d(int H, const CUtensorMap& mq, const CUtensorMap& mk, cons
     }
 }
 
+// Options of a tensor-core scoring launch.
+struct TcOpts {
+    bool units_ready = false;   // a set-up kernel already wrote the work units
+    int32_t planes = 1;         // 3: K holds three bf16 planes of fp32 keys, plane_rows rows apart
+    int64_t plane_rows = 0;
+    int32_t min_tiles = 8;      // key tiles per unit at least (tc_splits)
+};
+
+// Key tiles of a block map with whole 128-key tiles per block are contiguous: one tile load each.
+bool block_tiles(const ColMap& m) { return m.kind == kMapBlocks && m.block % 128 == 0; }
+
 // Tensor-core scores of launch rows [0, n_rows) (absolute [row_base, ...)) into
 // S[r * ld + c] for the eligible columns c < rows[r].ncols; column c is key
 // map(c) of the row's sequence.
 dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const TcSource& src, int H, int D,
                     const void* K, int64_t n_k, const int32_t* k_base, const ColMap& map, int32_t max_cols, float* S,
                     int64_t ld, TcUnit* units, int32_t* tile_base, uint32_t* status, cudaStream_t st,
-                    bool units_ready = false)
+                    const TcOpts& o = TcOpts{})
 {
     if (n_rows <= 0 || max_cols <= 0 || n_k <= 0) return DSA_OK;
     const int32_t TQ = tc_tile_rows(H);
     const int32_t tiles = tc_count_tiles(src.seq_off_host, src.n_seqs, row_base, n_rows, TQ);
     if (tiles == 0) return DSA_OK;
-    const int32_t splits = tc_splits(tiles, max_cols);
-    const bool gather = map.kind != kMapIdentity || map.offset != 0;
+    const int32_t splits = tc_splits(tiles, max_cols, o.min_tiles);
+    const bool btiles = block_tiles(map);
+    const bool gather = (map.kind != kMapIdentity || map.offset != 0) && !btiles;
+    const bool units_ready = o.units_ready;
     CUtensorMap mq, mk, mkg;
     if (!make_tile_map(&mq, src.Q, src.q_rows * H, D, 256) || !make_tile_map(&mk, K, n_k, D, 128) ||
         !make_tile_map(&mkg, K, n_k, D, 1))
@@ -537,6 +556,9 @@ dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const
     a.ld_s = ld;
     a.status = status;
     a.n_keys = n_k;
+    a.planes = o.planes;
+    a.plane_rows = o.plane_rows;
+    a.block_tiles = btiles ? 1 : 0;
     switch (D) {
     case 32: return launch_tc_d<32>(H, mq, mk, mkg, a, tiles * splits, n_acc, st);
     case 64: return launch_tc_d<64>(H, mq, mk, mkg, a, tiles * splits, n_acc, st);
@@ -762,6 +784,8 @@ struct HisaPlan {
     TcUnit* units;
     int32_t* tile_base;
     SelectSplit split;     // the token stage's select
+    uint32_t* planes;      // the pooled keys as three bf16 planes (one-pass step)
+    TcUnit* block_units;   // the block stage's scoring units (one-pass step)
 };
 
 std::vector<int32_t> iota_host(int32_t n)
@@ -769,6 +793,45 @@ std::vector<int32_t> iota_host(int32_t n)
     std::vector<int32_t> v(n + 1);
     for (int32_t i = 0; i <= n; ++i) v[i] = i;
     return v;
+}
+
+// Sizes of HISA's one-pass step (hisa_one_pass): pooled blocks, the block stage's query tiles
+// and key-range splits (units of one key tile of 128 blocks), and the token stage's splits
+// (units of at least two key tiles; every query is its own segment).
+struct HisaShape {
+    int64_t blocks;
+    int32_t max_mid;
+    int32_t tok_cols;
+    int32_t block_tiles;
+    int32_t block_splits;
+    int32_t token_splits;
+};
+
+HisaShape hisa_shape(const dsa_batch* b, const HostInfo& hi, int32_t B, int32_t keep)
+{
+    HisaShape h{};
+    for (int i = 0; i < b->num_seqs; ++i) h.blocks += (b->k_offsets_host[i + 1] - b->k_offsets_host[i] + B - 1) / B;
+    h.max_mid = std::max(0, (hi.max_k + B - 1) / B - 2);
+    h.tok_cols = (keep + 2) * B;
+    h.block_tiles = tc_count_tiles(b->q_offsets_host, b->num_seqs, 0, b->num_queries, tc_tile_rows(b->num_heads));
+    h.block_splits = tc_splits(h.block_tiles, h.max_mid, 1);
+    h.token_splits = tc_splits(b->num_queries, h.tok_cols, 2);
+    return h;
+}
+
+// Rows the register top-k takes (one CTA of up to 1024 threads, 16 columns each).
+constexpr int32_t kRegsMaxCols = 16384;
+
+// Whether a HISA call runs as the one-pass step: the sequences' tile offsets fit the set-up's
+// argument block, both stages' rows fit the register top-k, and both stages' scores fit the score
+// buffer at once.
+bool hisa_one_pass_ok(const dsa_batch* b, const HostInfo& hi, int32_t B, int32_t keep)
+{
+    const int32_t nq = b->num_queries;
+    if (nq <= 0 || b->num_seqs > kSetupMaxSeqs) return false;
+    const HisaShape h = hisa_shape(b, hi, B, keep);
+    if (h.max_mid > kRegsMaxCols || h.tok_cols > kRegsMaxCols || 3 * h.blocks > INT32_MAX) return false;
+    return chunk_rows(nq, score_ld(h.max_mid)) >= nq && chunk_rows(nq, score_ld(h.tok_cols)) >= nq;
 }
 
 size_t hisa_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, int32_t B, int32_t keep, HisaPlan* p)
@@ -795,6 +858,15 @@ size_t hisa_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k, 
     p->split.max_rows = split_rows_for(chunk_rows(nq, ld_tok));
     p->split.buf = c.take<uint64_t>(size_t(p->split.max_rows) * select_cap(k, (keep + 2) * B));
     if (base) p->split.ctr = split_counters(base);
+    if (hisa_one_pass_ok(b, hi, B, keep)) {
+        const HisaShape h = hisa_shape(b, hi, B, keep);
+        p->planes = c.take<uint32_t>(size_t(3) * h.blocks * b->head_dim / 2);
+        p->block_units = c.take<TcUnit>(size_t(h.block_tiles) * h.block_splits);
+        p->units = c.take<TcUnit>(size_t(nq) * h.token_splits);   // (replaces the chunked path's table)
+    } else {
+        p->planes = nullptr;
+        p->block_units = nullptr;
+    }
     return c.off;
 }
 
@@ -841,7 +913,7 @@ dsa_status dense_topk_one_launch(const dsa_batch* b, const HostInfo& hi, const T
     const int64_t ld = score_ld(hi.max_k);
     uint32_t* status = static_cast<uint32_t*>(ws);
     s = tc_score(p.rows, b->num_queries, 0, src, b->num_heads, b->head_dim, K, b->num_keys, b->k_offsets, ColMap{},
-                 hi.max_k, p.S, ld, p.units, p.tile_base, status, st, true);
+                 hi.max_k, p.S, ld, p.units, p.tile_base, status, st, TcOpts{true});
     if (s != DSA_OK) return s;
     return launch_select(p.rows, b->num_queries, hi.max_k, k, ColMap{}, p.S, ld, false, idx, k, scores, k, st, p.split);
 }
@@ -861,6 +933,135 @@ dsa_status refine_stage(const dsa_batch* b, const void* Q, const void* K, const 
     return tc_score_and_select(p.query_rows, b->num_queries, srf, b->num_heads, b->head_dim, K, b->num_keys,
                                b->k_offsets, m, C, p.S, p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k,
                                nullptr, st);
+}
+
+// The register top-k kernels, by row length (rows of at most kRegsMaxCols columns); smem: the
+// staged output row.
+template <template <int, int> class Launch, typename... Args>
+dsa_status launch_regs(int32_t max_cols, size_t smem, Args&&... args)
+{
+    if (max_cols <= 2048) return Launch<256, 8>::run(smem, args...);
+    if (max_cols <= 4096) return Launch<512, 8>::run(smem, args...);
+    if (max_cols <= 8192) return Launch<1024, 8>::run(smem, args...);
+    if (max_cols <= 12288) return Launch<1024, 12>::run(smem, args...);
+    return Launch<1024, 16>::run(smem, args...);
+}
+
+template <int NT, int R>
+struct RegsSelect {
+    static dsa_status run(size_t smem, int32_t n_rows, const SelectArgs& a, cudaStream_t st)
+    {
+        dsa_status s = set_smem(select_regs_kernel<NT, R>, smem);
+        if (s != DSA_OK) return s;
+        DSA_LAUNCH(kProfSelect, st, launch_pdl(latency_bound(n_rows), select_regs_kernel<NT, R>, n_rows, NT, smem, st, a));
+        return launched();
+    }
+};
+
+template <int NT, int R>
+struct RegsHisaBlocks {
+    static dsa_status run(size_t smem, int32_t n_rows, const SelectArgs& a, const HisaKeptArgs& h, cudaStream_t st)
+    {
+        dsa_status s = set_smem(hisa_block_select_kernel<NT, R>, smem);
+        if (s != DSA_OK) return s;
+        DSA_LAUNCH(kProfSelect, st, launch_pdl(latency_bound(n_rows), hisa_block_select_kernel<NT, R>, n_rows, NT, smem,
+                                               st, a, h));
+        return launched();
+    }
+};
+
+// HISA in one launch per stage (hisa_one_pass_ok): set-up (rows, block units, the pooled keys'
+// bf16 planes), block scores on the tensor cores, block top-`keep` fused with the kept blocks, the
+// token rows and the token units, token scores on the tensor cores (one tile load per kept block
+// when blocks are whole key tiles), token top-k: five launches, the later four programmatic.
+dsa_status hisa_one_pass(const dsa_batch* b, const HostInfo& hi, const void* Q, const void* K, const float* W,
+                         const float* pooled, int32_t k, int32_t B, int32_t keep, int32_t* idx, int32_t* kept,
+                         const HisaPlan& p, void* ws, cudaStream_t st)
+{
+    const int32_t nq = b->num_queries, H = b->num_heads, D = b->head_dim;
+    const HisaShape h = hisa_shape(b, hi, B, keep);
+    uint32_t* status = static_cast<uint32_t*>(ws);
+    g_status = status;
+    HisaSetupArgs a{};
+    a.q_off = b->q_offsets;
+    a.k_off = b->k_offsets;
+    a.q_pos = b->q_pos;
+    a.pooled = pooled;
+    a.planes = p.planes;
+    a.rows = p.block_rows;
+    a.units = p.block_units;
+    a.query_off = p.query_off;
+    a.header = status;
+    a.header_words = (int32_t)(kHeaderBytes / 4);
+    a.n_seqs = b->num_seqs;
+    a.n_q = nq;
+    a.B = B;
+    a.TQ = tc_tile_rows(H);
+    int32_t tiles = 0, blocks = 0;
+    for (int i = 0; i < b->num_seqs; ++i) {
+        a.tile_base[i] = tiles;
+        a.block_base[i] = blocks;
+        tiles += (b->q_offsets_host[i + 1] - b->q_offsets_host[i] + a.TQ - 1) / a.TQ;
+        blocks += (b->k_offsets_host[i + 1] - b->k_offsets_host[i] + B - 1) / B;
+    }
+    a.tile_base[b->num_seqs] = tiles;
+    a.block_base[b->num_seqs] = blocks;
+    a.splits = h.block_splits;
+    a.n_units = h.block_tiles * h.block_splits;
+    a.n_pairs = int64_t(blocks) * D / 2;
+    a.row_ctas = (std::max(nq + 1, a.n_units) + 255) / 256;
+    const int split_ctas = (int)std::min<int64_t>(2 * 148, (a.n_pairs + 255) / 256);
+    DSA_LAUNCH(kProfSetup, st, launch_pdl(false, hisa_setup_tc_kernel, a.row_ctas + split_ctas, 256, 0, st, a));
+    dsa_status s = launched();
+    if (s != DSA_OK) return s;
+
+    // Coarse stage: the middle blocks' pooled keys as three bf16 planes on the tensor cores.
+    const TcSource bsrc{Q, nq, W, b->q_offsets, b->q_offsets_host, b->num_seqs};
+    const int64_t ld_blk = score_ld(h.max_mid), ld_tok = score_ld(h.tok_cols);
+    TcOpts ob;
+    ob.units_ready = true;
+    ob.planes = 3;
+    ob.plane_rows = blocks;
+    ob.min_tiles = 1;
+    s = tc_score(p.block_rows, nq, 0, bsrc, H, D, p.planes, 3 * int64_t(blocks), nullptr, ColMap{}, h.max_mid, p.S,
+                 ld_blk, p.block_units, p.tile_base, status, st, ob);
+    if (s != DSA_OK) return s;
+    SelectArgs sa{};
+    sa.rows = p.block_rows;
+    sa.n_rows = nq;
+    sa.k = keep;
+    sa.map = identity_map(1);   // column c is middle block c + 1
+    sa.S = p.S;
+    sa.ld_s = ld_blk;
+    sa.status = status;
+    const HisaKeptArgs ka{b->q_pos, b->k_offsets, B, keep, h.token_splits, 0, kept, p.token_rows, p.units};
+    if ((s = launch_regs<RegsHisaBlocks>(h.max_mid, size_t(keep) * 4, nq, sa, ka, st)) != DSA_OK) return s;
+
+    // Fine stage: the indexer over the tokens of the kept blocks, then the top k.
+    ColMap m{};
+    m.kind = kMapBlocks;
+    m.block = B;
+    m.list = kept;
+    m.list_ld = keep + 2;
+    const std::vector<int32_t> qoff = iota_host(nq);
+    const TcSource tsrc{Q, nq, W, p.query_off, qoff.data(), nq};
+    TcOpts ot;
+    ot.units_ready = true;
+    ot.min_tiles = 2;
+    s = tc_score(p.token_rows, nq, 0, tsrc, H, D, K, b->num_keys, b->k_offsets, m, h.tok_cols, p.S, ld_tok, p.units,
+                 p.tile_base, status, st, ot);
+    if (s != DSA_OK) return s;
+    SelectArgs ta{};
+    ta.rows = p.token_rows;
+    ta.n_rows = nq;
+    ta.k = k;
+    ta.map = m;
+    ta.S = p.S;
+    ta.ld_s = ld_tok;
+    ta.status = status;
+    ta.out_idx = idx;
+    ta.ld_idx = k;
+    return launch_regs<RegsSelect>(h.tok_cols, size_t(k) * 4, nq, ta, st);
 }
 
 }  // namespace
@@ -1330,6 +1531,7 @@ dsa_status hisa_index(const dsa_batch* b, const void* Q, const void* K, const fl
     g_status = static_cast<uint32_t*>(ws);   // hisa_setup_kernel clears the header
     const int H = b->num_heads, D = b->head_dim;
     int32_t* kept = kept_out ? kept_out : p.kept;
+    if (p.planes) return hisa_one_pass(b, hi, Q, K, W, pooled, k, B, keep, idx, kept, p, ws, st);
     const unsigned g = (nq + 255) / 256;
 
     DSA_LAUNCH(kProfSetup, st, hisa_setup_kernel<<<(nq + 256) / 256, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos,
@@ -1359,7 +1561,7 @@ dsa_status hisa_index(const dsa_batch* b, const void* Q, const void* K, const fl
                                               p.token_rows, p.units));
         if ((s = launched()) != DSA_OK) return s;
         s = tc_score(p.token_rows, nq, 0, src, H, D, K, b->num_keys, b->k_offsets, m, tok_cols, p.S, ld_tok, p.units,
-                     p.tile_base, static_cast<uint32_t*>(ws), st, true);
+                     p.tile_base, static_cast<uint32_t*>(ws), st, TcOpts{true});
         if (s != DSA_OK) return s;
         return launch_select(p.token_rows, nq, tok_cols, k, m, p.S, ld_tok, false, idx, k, nullptr, 0, st, p.split);
     }

@@ -26,6 +26,11 @@
 //   warps 10-11 more producers of gathered tiles (idle for contiguous ones)
 // The two accumulators are handed back and forth between MMA and epilogue
 // with mbarriers, so the MMAs into one overlap the epilogue of the other.
+// Keys kept in fp32 (HISA's pooled block keys) are scored as three bf16 planes:
+// each value v is hi + mid + lo exactly (each part the leading 8 significant
+// bits of what remains), the three tiles of a key tile pass through the ring
+// one after another and accumulate into the same TMEM columns, so the sum
+// q . hi + q . mid + q . lo is the fp32 dot product up to accumulation order.
 // Every wait is bounded (1 s); a wait that runs out records an error in the
 // workspace status word and the CTA drains its copies and MMAs and exits.
 #pragma once
@@ -52,8 +57,12 @@ struct TcArgs {
     int64_t ld_s;
     uint32_t* status;
     int32_t n_stages;
-    int32_t pad_;
+    int32_t planes;          // 1, or 3: a key tile is the sum of three bf16 tiles (hi, mid, lo) plane_rows apart
     int64_t n_keys;          // rows of K (checked builds verify every gathered key row against it)
+    int64_t plane_rows;
+    int32_t block_tiles;     // contiguous launches: column c is key list[c / block] * block + c % block, with
+                             // whole 128-key tiles per block (block a multiple of 128): one tile load each
+    int32_t pad2_;
 };
 
 template <int D, int H>
@@ -104,13 +113,19 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, uint32_t
     }
 }
 
-// GATHER: the unit's key tiles are gathered through the column map (a.gather == 1).  The two
-// cases are compiled apart, so contiguous tiles keep the single-producer code.
-template <int D, int H, bool GATHER>
-__global__ void __launch_bounds__(GATHER ? kTcThreads : kTcThreadsTiles, 1)
+// MODE kTcTiles: contiguous key tiles; kTcGather: the unit's key tiles are gathered through the
+// column map (a.gather == 1); kTcBlocks: contiguous tiles at computed rows, the three planes of
+// fp32 keys (a.planes) or whole 128-key tiles of a block map (a.block_tiles).  The cases are
+// compiled apart, so the dense scan keeps the leanest producer and MMA-issuer loops.
+enum : int { kTcTiles = 0, kTcGather = 1, kTcBlocks = 2 };
+
+template <int D, int H, int MODE>
+__global__ void __launch_bounds__(MODE == kTcGather ? kTcThreads : kTcThreadsTiles, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmKg, TcArgs a)
 {
+    constexpr bool GATHER = MODE == kTcGather;
+    constexpr bool EXT = MODE == kTcBlocks;
     using SH = TcShape<D, H>;
     constexpr int NP = GATHER ? kTcProducers : 1;   // producers with a full barrier per stage
     constexpr int NQA = SH::NQA;
@@ -191,13 +206,14 @@ __global__ void __launch_bounds__(GATHER ? kTcThreads : kTcThreadsTiles, 1)
         uint64_t* my_full = full + pw * n_stages;
         // the columns of the unit that exist (tiles past them read column 0's key)
         int ncmax = 0, list = 0;
+        if (GATHER || (EXT && a.block_tiles)) list = a.rows[u.row0].list;
         if (GATHER) {
-            list = a.rows[u.row0].list;
             for (int j = lane; j < u.nrows; j += 32) ncmax = max(ncmax, a.rows[u.row0 + j].ncols);
             ncmax = __reduce_max_sync(0xffffffffu, ncmax);
         }
         const RowDesc first{0, 0, 0, list};   // map_col reads only the list row
-        const int32_t* lrow = GATHER && a.map.kind != kMapIdentity ? a.map.list + (int64_t)list * a.map.list_ld : nullptr;
+        const int32_t* lrow = (GATHER || (EXT && a.block_tiles)) && a.map.kind != kMapIdentity
+                                  ? a.map.list + (int64_t)list * a.map.list_ld : nullptr;
         const bool list4 = a.map.kind == kMapList && (reinterpret_cast<uintptr_t>(lrow) & 15) == 0;
         const bool block4 = a.map.kind == kMapBlocks && (a.map.block & 3) == 0;
         // Key rows of this lane's four rows (columns c0 .. c0+3) of tile i: one 16-byte list load,
@@ -225,14 +241,30 @@ __global__ void __launch_bounds__(GATHER ? kTcThreads : kTcThreadsTiles, 1)
         int stage = 0;
         uint32_t phase = 0;
         int issued = 0;
-        for (int i = 0; i < nkt; ++i) {
+        const int planes = EXT ? a.planes : 1;
+        int32_t blk = 0;   // block tiles: lane l holds the block of tile i0 + l
+        for (int e = 0; e < nkt * planes; ++e) {
+            const int i = EXT ? e / planes : e, pl = EXT ? e - i * planes : 0;
             int ok = 1;
             if (lane == 0) ok = tc_wait(&empty[stage], phase ^ 1u, a.status, 1, abort_flag) ? 1 : 0;
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             if constexpr (!GATHER) {
+                int krow;
+                if (EXT && a.block_tiles) {
+                    if ((i & 31) == 0 && pl == 0) {   // the next 32 tiles' blocks, one load per lane
+                        const int c = (u.kt0 + i + lane) * 128;
+                        blk = i + lane < nkt ? __ldg(lrow + c / a.map.block) : 0;
+                    }
+                    const int c0 = (u.kt0 + i) * 128;
+                    krow = krow0 + __shfl_sync(0xffffffffu, blk, i & 31) * a.map.block + c0 % a.map.block;
+                    if (!DSA_CHECK(krow >= 0 && krow < a.n_keys, a.status, 102)) krow = 0;   // a block's first key row
+                } else if (EXT) {
+                    krow = krow0 + (u.kt0 + i) * 128 + (int)(pl * a.plane_rows);
+                } else {
+                    krow = krow0 + (u.kt0 + i) * 128;
+                }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&my_full[stage], SH::KTILE);
-                    const int krow = krow0 + (u.kt0 + i) * 128;
                     for (int bx = 0; bx < SH::NBOX; ++bx) {
                         if (a.keep_keys)
                             tma_load_2d_hint(sK + stage * SH::KTILE + bx * SH::KBOX, &tmK, bx * SH::BOXC, krow,
@@ -279,7 +311,9 @@ __global__ void __launch_bounds__(GATHER ? kTcThreads : kTcThreadsTiles, 1)
                 int stage = 0;
                 uint32_t phase = 0;
                 uint32_t tph[2] = {0, 0};
-                for (int i = 0; i < nkt && !*abort_flag; ++i) {
+                const int planes = EXT ? a.planes : 1;
+                for (int e = 0; e < nkt * planes && !*abort_flag; ++e) {
+                    const int i = EXT ? e / planes : e, pl = EXT ? e - i * planes : 0;
                     bool landed = true;
                     for (int p = 0; p < NP && landed; ++p)
                         landed = tc_wait(&full[p * n_stages + stage], phase, a.status, 3, abort_flag);
@@ -288,8 +322,10 @@ __global__ void __launch_bounds__(GATHER ? kTcThreads : kTcThreadsTiles, 1)
                     for (int qb = 0; qb < n_acc; ++qb) {
                         // one query block: the two accumulators alternate tile by tile
                         const int slot = n_acc == 1 ? (i & 1) : qb;
-                        if (!tc_wait(&tempty[slot], tph[slot] ^ 1u, a.status, 4, abort_flag)) break;
-                        tc_fence_after();
+                        if (pl == 0) {   // a tile's first plane starts the accumulator afresh
+                            if (!tc_wait(&tempty[slot], tph[slot] ^ 1u, a.status, 4, abort_flag)) break;
+                            tc_fence_after();
+                        }
                         const uint32_t d = tmem + slot * 256;
 #pragma unroll
                         for (int kk = 0; kk < SH::KSTEPS; ++kk) {
@@ -299,10 +335,12 @@ __global__ void __launch_bounds__(GATHER ? kTcThreads : kTcThreadsTiles, 1)
                                 smem_desc_kmajor(smem_u32(sK + stage * SH::KTILE + bx * SH::KBOX) + ko, SH::ROWB);
                             const uint64_t bd =
                                 smem_desc_kmajor(smem_u32(sQ + qb * SH::QACC + bx * SH::QBOX) + ko, SH::ROWB);
-                            tc_mma(d, ad, bd, idesc[qb], kk > 0 ? 1u : 0u);
+                            tc_mma(d, ad, bd, idesc[qb], kk > 0 || pl > 0 ? 1u : 0u);
                         }
-                        tc_commit(&tfull[slot]);
-                        tph[slot] ^= 1u;
+                        if (pl == planes - 1) {
+                            tc_commit(&tfull[slot]);
+                            tph[slot] ^= 1u;
+                        }
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == n_stages) { stage = 0; phase ^= 1u; }

@@ -103,6 +103,35 @@ __device__ __forceinline__ void block_key_range(uint32_t& lo, uint32_t& hi, uint
     for (int w = 1; w < kSelWarps; ++w) { lo = min(lo, scratch[w]); hi = max(hi, scratch[kSelWarps + w]); }
 }
 
+// Run by one warp after a radix pass: finds the bin of the 256-bin histogram that holds rank krem
+// (1 = largest) and writes out[0] = the bin, out[1] = the keys in the bins above it, out[2] = 1 when
+// the bin's keys are all taken (rank krem is its lowest key).
+__device__ __forceinline__ void radix_pick(const uint32_t* hist, int krem, uint32_t* out)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t c[8], tot = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) { c[b] = hist[8 * lane + b]; tot += c[b]; }
+    uint32_t incl = tot;   // keys in the digits of lanes >= this lane
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += x;
+    }
+    const uint32_t above = incl - tot;
+    if (above < (uint32_t)krem && (uint32_t)krem <= incl) {
+        uint32_t acc = above;
+        int b = 7;
+        for (; b > 0; --b) {
+            if (acc + c[b] >= (uint32_t)krem) break;
+            acc += c[b];
+        }
+        out[0] = 8 * lane + b;
+        out[1] = acc;
+        out[2] = acc + c[b] == (uint32_t)krem;   // the whole bin is taken
+    }
+}
+
 // Exact rank selection among `count` keys given by get(i): returns the key T
 // holding rank `krem` (1 = largest) and, in krem, how many keys equal to T
 // that rank reaches.  Digits are taken from (key - min), starting at the
@@ -121,7 +150,7 @@ __device__ __forceinline__ uint32_t radix_select_in(Get get, int count, int& kre
 {
     constexpr int kSelThreads = NT;
     constexpr int kSelWarps = NT / 32;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5;
     int top = 32 - __clz(hi - lo);   // bits of (key - lo) still undecided
     const int stop = stop_bits > 0 ? max(top - stop_bits, 0) : 0;
     uint32_t prefix = 0;             // decided high bits of (T - lo)
@@ -135,29 +164,7 @@ __device__ __forceinline__ uint32_t radix_select_in(Get get, int count, int& kre
             if (((rel >> 1) >> (top - 1)) == prefix) atomicAdd(&hist[(rel >> shift) & ((1u << width) - 1u)], 1u);
         }
         __syncthreads();
-        if (warp == 0) {
-            uint32_t c[8], tot = 0;
-#pragma unroll
-            for (int b = 0; b < 8; ++b) { c[b] = hist[8 * lane + b]; tot += c[b]; }
-            uint32_t incl = tot;   // keys in the digits of lanes >= this lane
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t x = __shfl_down_sync(0xffffffffu, incl, o);
-                if (lane + o < 32) incl += x;
-            }
-            const uint32_t above = incl - tot;
-            if (above < (uint32_t)krem && (uint32_t)krem <= incl) {
-                uint32_t acc = above;
-                int b = 7;
-                for (; b > 0; --b) {
-                    if (acc + c[b] >= (uint32_t)krem) break;
-                    acc += c[b];
-                }
-                scratch[2 * kSelWarps] = 8 * lane + b;
-                scratch[2 * kSelWarps + 1] = acc;
-                scratch[2 * kSelWarps + 2] = acc + c[b] == (uint32_t)krem;   // the whole bin is taken
-            }
-        }
+        if (warp == 0) radix_pick(hist, krem, scratch + 2 * kSelWarps);
         __syncthreads();
         prefix = (prefix << width) | scratch[2 * kSelWarps];
         krem -= (int)scratch[2 * kSelWarps + 1];

@@ -296,6 +296,102 @@ __global__ void hisa_setup_kernel(const int32_t* q_off, const int32_t* k_off, co
     rows[t] = RowDesc{t, b, last > 1 ? last - 1 : 0, t};
 }
 
+// The three bf16 planes of an fp32 value: v = hi + mid + lo exactly.  hi is v with its low 16
+// mantissa bits cleared; the remainder v - hi (exact: at most 16 significant bits) is split the
+// same way, and what is left after that has at most 8 significant bits, so it is a bf16 itself.
+__device__ __forceinline__ void split_bf16x3(float v, uint32_t& hi, uint32_t& mid, uint32_t& lo)
+{
+    const uint32_t hb = __float_as_uint(v) & 0xffff0000u;
+    const float r1 = v - __uint_as_float(hb);
+    const uint32_t mb = __float_as_uint(r1) & 0xffff0000u;
+    const float r2 = r1 - __uint_as_float(mb);
+    hi = hb >> 16;
+    mid = mb >> 16;
+    lo = __float_as_uint(r2) >> 16;
+}
+
+// HISA's set-up for a block stage on the tensor cores, one launch.  CTAs [0, row_ctas): the
+// workspace header cleared, query_off = 0..n_q, one block row per query (its middle blocks
+// 1 .. last - 1 as columns 0 .. last - 2) and the block-scoring work units (as dense_setup_kernel's:
+// tiles of TQ queries of one sequence, each tile's middle-block columns split `splits` ways; the key
+// row of column 0 is the sequence's block 1 in plane 0).  The other CTAs split the pooled fp32 keys
+// into the three bf16 planes the scoring kernel reads (plane p at rows p * n_blocks).
+struct HisaSetupArgs {
+    const int32_t* q_off;
+    const int32_t* k_off;
+    const int32_t* q_pos;
+    const float* pooled;        // [n_blocks, D]
+    uint32_t* planes;           // [3, n_blocks, D] bf16, as pairs
+    RowDesc* rows;
+    TcUnit* units;
+    int32_t* query_off;
+    uint32_t* header;           // zeroed: header_words words
+    int64_t n_pairs;            // n_blocks * D / 2
+    int32_t header_words;
+    int32_t n_seqs;
+    int32_t n_q;
+    int32_t B;
+    int32_t TQ;
+    int32_t splits;
+    int32_t n_units;
+    int32_t row_ctas;
+    int32_t tile_base[kSetupMaxSeqs + 1];    // first tile of each sequence
+    int32_t block_base[kSetupMaxSeqs + 1];   // first pooled block of each sequence
+};
+
+__device__ __forceinline__ int32_t hisa_mid_count(int32_t pos, int32_t L, int32_t B)
+{
+    const int n = eligible_count(pos, L);
+    const int last = n > 0 ? (n - 1) / B : 0;
+    return last > 1 ? last - 1 : 0;
+}
+
+__global__ void hisa_setup_tc_kernel(const __grid_constant__ HisaSetupArgs a)
+{
+    grid_dep_launch();   // the scoring kernel may set up; it waits for this grid before reading units
+    if ((int)blockIdx.x >= a.row_ctas) {
+        const int64_t stride = (int64_t)(gridDim.x - a.row_ctas) * blockDim.x;
+        const int64_t plane = a.n_pairs;   // 32-bit words per plane
+        const float2* src = reinterpret_cast<const float2*>(a.pooled);
+        for (int64_t i = (int64_t)(blockIdx.x - a.row_ctas) * blockDim.x + threadIdx.x; i < a.n_pairs; i += stride) {
+            const float2 v = __ldg(src + i);
+            uint32_t h0, m0, l0, h1, m1, l1;
+            split_bf16x3(v.x, h0, m0, l0);
+            split_bf16x3(v.y, h1, m1, l1);
+            a.planes[i] = h0 | (h1 << 16);
+            a.planes[plane + i] = m0 | (m1 << 16);
+            a.planes[2 * plane + i] = l0 | (l1 << 16);
+        }
+        return;
+    }
+    const int gid = blockIdx.x * blockDim.x + threadIdx.x;
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < a.header_words; i += blockDim.x) a.header[i] = 0u;
+    if (gid <= a.n_q) a.query_off[gid] = gid;
+    if (gid < a.n_q) {
+        const int b = find_seq(a.q_off, a.n_seqs, gid);
+        a.rows[gid] = RowDesc{gid, b, hisa_mid_count(a.q_pos[gid], a.k_off[b + 1] - a.k_off[b], a.B), gid};
+    }
+    if (gid < a.n_units) {
+        const int tau = gid / a.splits, s = gid % a.splits;
+        int lo = 0, hi = a.n_seqs - 1;   // the sequence whose tiles hold tile tau
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (a.tile_base[mid] <= tau) lo = mid; else hi = mid - 1;
+        }
+        const int b = lo;
+        const int q0 = a.q_off[b], nq = a.q_off[b + 1] - q0;
+        const int jj = tau - a.tile_base[b];
+        const int r0 = q0 + jj * a.TQ;
+        const int nr = min(a.TQ, nq - jj * a.TQ);
+        const int L = a.k_off[b + 1] - a.k_off[b];
+        int maxnc = 0;
+        for (int r = r0; r < r0 + nr; ++r) maxnc = max(maxnc, hisa_mid_count(a.q_pos[r], L, a.B));
+        const int nkt = (maxnc + 127) / 128;
+        a.units[gid] = TcUnit{r0, nr, nkt * s / a.splits, nkt * (s + 1) / a.splits, r0, a.block_base[b] + 1, {0, 0}};
+    }
+}
+
 // Kept blocks of query t: block 0, the selected middle blocks (ascending,
 // -1 padded), and the query's own block; then the token row over them.
 __global__ void hisa_kept_kernel(const RowDesc* block_rows, const int32_t* mid, int32_t keep,

@@ -219,11 +219,22 @@ def test_hisa_pool_integer_exact():
     assert np.array_equal(pooled[full].astype(np.float64), ref[full])
 
 
-@pytest.mark.parametrize("B,keep", [(64, 3), (128, 1), (64, 40)])
+@pytest.mark.parametrize("B,keep", [(64, 3), (128, 1), (64, 40), (128, 4), (256, 2)])
 def test_hisa_integer_exact(B, keep):
     b = workloads.ragged(9, [3, 2, 4], [1500, 700, 129], H=4, d=32, k=100, integer=True, pos_mode="random")
     idx, kept, _ = Dev(b).hisa(100, B, keep)
     ref = oracle.hisa(b, B, keep, 100)
+    check_exact_sets(kept, ref["kept"], "kept")
+    check_exact_sets(idx, ref["idx"], "idx")
+
+
+def test_hisa_many_sequences_exact():
+    """More sequences than the one-pass set-up takes (480): the step falls back to the staged path
+    (CUDA-core block scores, streaming selects); 490 one-query sequences, integer inputs, exact."""
+    lens = [200 + 37 * (i % 13) for i in range(490)]
+    b = workloads.ragged(12, [1] * 490, lens, H=4, d=32, k=40, integer=True, pos_mode="random")
+    idx, kept, _ = Dev(b).hisa(40, 64, 2)
+    ref = oracle.hisa(b, 64, 2, 40)
     check_exact_sets(kept, ref["kept"], "kept")
     check_exact_sets(idx, ref["idx"], "idx")
 
@@ -270,6 +281,15 @@ def test_hisa_bf16_needles():
     b = workloads.hisa_decode(seed=41, B=2, L=40000, n_mtp=2, H=64, d=128, k=512, block=128, keep=16,
                               n_needles=6)
     check_hisa_bf16(b, 512, 128, 16)
+
+
+@pytest.mark.parametrize("keep", [40, 100])
+def test_hisa_bf16_long_token_rows(keep):
+    """Token rows of 5376 and 13056 columns (40 and 100 kept middle blocks of 128): the longer
+    register top-k shapes."""
+    b = workloads.hisa_decode(seed=43, B=2, L=20000, n_mtp=2, H=64, d=128, k=2048, block=128, keep=keep,
+                              n_needles=4)
+    check_hisa_bf16(b, 2048, 128, keep)
 
 
 def test_full_size_hisa_256k():
