@@ -240,7 +240,11 @@ dsa_status pivot_refine_candidates(const dsa_batch* batch, const void* Q, const 
  * sequence), the blocks strictly between block 0 and `last` are scored with
  * the indexer formula against their pooled key; block 0, block `last` and the
  * `keep` best middle blocks are kept; the indexer then ranks every eligible
- * token of the kept blocks and returns its top k.
+ * token of the kept blocks and returns its top k.  Block scores take the fp32
+ * pooled key exactly (as the sum of three bf16 parts) with fp32 accumulation.
+ * The workspace includes a bf16 copy of the pooled keys (6 bytes per element)
+ * when every stage runs in one launch (at most 480 sequences, rows of at most
+ * 16,384 blocks and kept tokens).
  * idx [n_q, k]; kept [n_q, keep+2] int32 or NULL (ascending, -1 padded).
  * Requires block in {64, 128, 256}, 1 <= keep <= 256.
  */
