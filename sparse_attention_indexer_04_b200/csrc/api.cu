@@ -289,6 +289,29 @@ dsa_status set_smem(Kern kern, size_t smem)
                : DSA_ERR_CUDA;
 }
 
+// The register top-k kernels, by row length (rows of at most 16,384 columns); smem: the staged
+// output row.
+template <template <int, int> class Launch, typename... Args>
+dsa_status launch_regs(int32_t max_cols, size_t smem, Args&&... args)
+{
+    if (max_cols <= 2048) return Launch<256, 8>::run(smem, args...);
+    if (max_cols <= 4096) return Launch<512, 8>::run(smem, args...);
+    if (max_cols <= 8192) return Launch<1024, 8>::run(smem, args...);
+    if (max_cols <= 12288) return Launch<1024, 12>::run(smem, args...);
+    return Launch<1024, 16>::run(smem, args...);
+}
+
+template <int NT, int R>
+struct RegsSelect {
+    static dsa_status run(size_t smem, int32_t n_rows, const SelectArgs& a, cudaStream_t st)
+    {
+        dsa_status s = set_smem(select_regs_kernel<NT, R>, smem);
+        if (s != DSA_OK) return s;
+        DSA_LAUNCH(kProfSelect, st, launch_pdl(latency_bound(n_rows), select_regs_kernel<NT, R>, n_rows, NT, smem, st, a));
+        return launched();
+    }
+};
+
 // n_rows_dev (optional): only rows below the count a kernel wrote there are ranked, and each
 // writes output row rows[r].qrow (the one-CTA-per-row kernel only).
 dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, int32_t k, const ColMap& map,
@@ -459,7 +482,7 @@ int32_t tc_unit_capacity(const TcSource& src, int32_t n_rows, int32_t chunk, int
 
 template <int D, int H>
 dsa_status launch_tc_shape(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mkg, const TcArgs& a,
-                           int32_t n_units, int n_acc, cudaStream_t st)
+                           const DenseSetupArgs& su, int32_t n_units, int n_acc, cudaStream_t st)
 {
     using SH = TcShape<D, H>;
     const int budget = 232448;
@@ -474,31 +497,31 @@ dsa_status launch_tc_shape(const CUtensorMap& mq, const CUtensorMap& mk, const C
     if (a.gather) {
         if ((s = set_smem(score_tc_kernel<D, H, kTcGather>, smem)) != DSA_OK) return s;
         DSA_LAUNCH(kProfScoreTc, st, launch_pdl(latency_bound(n_units), score_tc_kernel<D, H, kTcGather>, n_units,
-                                                kTcThreads, smem, st, mq, mk, mkg, args));
+                                                kTcThreads, smem, st, mq, mk, mkg, args, su));
     } else if (a.planes > 1 || a.block_tiles) {
         if ((s = set_smem(score_tc_kernel<D, H, kTcBlocks>, smem)) != DSA_OK) return s;
         DSA_LAUNCH(kProfScoreTc, st, launch_pdl(latency_bound(n_units), score_tc_kernel<D, H, kTcBlocks>, n_units,
-                                                kTcThreadsTiles, smem, st, mq, mk, mkg, args));
+                                                kTcThreadsTiles, smem, st, mq, mk, mkg, args, su));
     } else {
         if ((s = set_smem(score_tc_kernel<D, H, kTcTiles>, smem)) != DSA_OK) return s;
         DSA_LAUNCH(kProfScoreTc, st, launch_pdl(latency_bound(n_units), score_tc_kernel<D, H, kTcTiles>, n_units,
-                                                kTcThreadsTiles, smem, st, mq, mk, mkg, args));
+                                                kTcThreadsTiles, smem, st, mq, mk, mkg, args, su));
     }
     return launched();
 }
 
 template <int D>
 dsa_status launch_tc_d(int H, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mkg, const TcArgs& a,
-                       int32_t n_units, int n_acc, cudaStream_t st)
+                       const DenseSetupArgs& su, int32_t n_units, int n_acc, cudaStream_t st)
 {
     switch (H) {
-    case 1: return launch_tc_shape<D, 1>(mq, mk, mkg, a, n_units, n_acc, st);
-    case 2: return launch_tc_shape<D, 2>(mq, mk, mkg, a, n_units, n_acc, st);
-    case 4: return launch_tc_shape<D, 4>(mq, mk, mkg, a, n_units, n_acc, st);
-    case 8: return launch_tc_shape<D, 8>(mq, mk, mkg, a, n_units, n_acc, st);
-    case 16: return launch_tc_shape<D, 16>(mq, mk, mkg, a, n_units, n_acc, st);
-    case 32: return launch_tc_shape<D, 32>(mq, mk, mkg, a, n_units, n_acc, st);
-    default: return launch_tc_shape<D, 64>(mq, mk, mkg, a, n_units, n_acc, st);
+    case 1: return launch_tc_shape<D, 1>(mq, mk, mkg, a, su, n_units, n_acc, st);
+    case 2: return launch_tc_shape<D, 2>(mq, mk, mkg, a, su, n_units, n_acc, st);
+    case 4: return launch_tc_shape<D, 4>(mq, mk, mkg, a, su, n_units, n_acc, st);
+    case 8: return launch_tc_shape<D, 8>(mq, mk, mkg, a, su, n_units, n_acc, st);
+    case 16: return launch_tc_shape<D, 16>(mq, mk, mkg, a, su, n_units, n_acc, st);
+    case 32: return launch_tc_shape<D, 32>(mq, mk, mkg, a, su, n_units, n_acc, st);
+    default: return launch_tc_shape<D, 64>(mq, mk, mkg, a, su, n_units, n_acc, st);
     }
 }
 
@@ -508,6 +531,7 @@ struct TcOpts {
     int32_t planes = 1;         // 3: K holds three bf16 planes of fp32 keys, plane_rows rows apart
     int64_t plane_rows = 0;
     int32_t min_tiles = 8;      // key tiles per unit at least (tc_splits)
+    const DenseSetupArgs* own_setup = nullptr;   // dense launches of one wave: the kernel's own set-up
 };
 
 // Key tiles of a block map with whole 128-key tiles per block are contiguous: one tile load each.
@@ -559,10 +583,12 @@ dsa_status tc_score(const RowDesc* rows, int32_t n_rows, int32_t row_base, const
     a.planes = o.planes;
     a.plane_rows = o.plane_rows;
     a.block_tiles = btiles ? 1 : 0;
+    static const DenseSetupArgs kNoSetup{};
+    const DenseSetupArgs& su = o.own_setup ? *o.own_setup : kNoSetup;
     switch (D) {
-    case 32: return launch_tc_d<32>(H, mq, mk, mkg, a, tiles * splits, n_acc, st);
-    case 64: return launch_tc_d<64>(H, mq, mk, mkg, a, tiles * splits, n_acc, st);
-    default: return launch_tc_d<128>(H, mq, mk, mkg, a, tiles * splits, n_acc, st);
+    case 32: return launch_tc_d<32>(H, mq, mk, mkg, a, su, tiles * splits, n_acc, st);
+    case 64: return launch_tc_d<64>(H, mq, mk, mkg, a, su, tiles * splits, n_acc, st);
+    default: return launch_tc_d<128>(H, mq, mk, mkg, a, su, tiles * splits, n_acc, st);
     }
 }
 
@@ -905,15 +931,22 @@ dsa_status dense_topk_one_launch(const dsa_batch* b, const HostInfo& hi, const T
     a.tile_base[b->num_seqs] = tiles;
     a.splits = tc_splits(tiles, hi.max_k);   // as tc_score derives it
     a.n_units = tiles * a.splits;
-    const int grid = (std::max(a.n_q, a.n_units) + 255) / 256;
-    // a plain launch: it starts once the stream's earlier work (which may use this workspace) is done
-    DSA_LAUNCH(kProfSetup, st, launch_pdl(false, dense_setup_kernel, grid, 256, 0, st, a));
-    dsa_status s = launched();
-    if (s != DSA_OK) return s;
+    TcOpts o;
+    o.units_ready = true;
+    dsa_status s;
+    if (a.n_units <= 148) {
+        // one wave (decode): the scoring kernel sets itself up (every query row is in some unit's tile)
+        o.own_setup = &a;
+    } else {
+        const int grid = (std::max(a.n_q, a.n_units) + 255) / 256;
+        // a plain launch: it starts once the stream's earlier work (which may use this workspace) is done
+        DSA_LAUNCH(kProfSetup, st, launch_pdl(false, dense_setup_kernel, grid, 256, 0, st, a));
+        if ((s = launched()) != DSA_OK) return s;
+    }
     const int64_t ld = score_ld(hi.max_k);
     uint32_t* status = static_cast<uint32_t*>(ws);
     s = tc_score(p.rows, b->num_queries, 0, src, b->num_heads, b->head_dim, K, b->num_keys, b->k_offsets, ColMap{},
-                 hi.max_k, p.S, ld, p.units, p.tile_base, status, st, TcOpts{true});
+                 hi.max_k, p.S, ld, p.units, p.tile_base, status, st, o);
     if (s != DSA_OK) return s;
     return launch_select(p.rows, b->num_queries, hi.max_k, k, ColMap{}, p.S, ld, false, idx, k, scores, k, st, p.split);
 }
@@ -934,29 +967,6 @@ dsa_status refine_stage(const dsa_batch* b, const void* Q, const void* K, const 
                                b->k_offsets, m, C, p.S, p.units, p.tile_base, static_cast<uint32_t*>(ws), k, idx, k,
                                nullptr, st);
 }
-
-// The register top-k kernels, by row length (rows of at most kRegsMaxCols columns); smem: the
-// staged output row.
-template <template <int, int> class Launch, typename... Args>
-dsa_status launch_regs(int32_t max_cols, size_t smem, Args&&... args)
-{
-    if (max_cols <= 2048) return Launch<256, 8>::run(smem, args...);
-    if (max_cols <= 4096) return Launch<512, 8>::run(smem, args...);
-    if (max_cols <= 8192) return Launch<1024, 8>::run(smem, args...);
-    if (max_cols <= 12288) return Launch<1024, 12>::run(smem, args...);
-    return Launch<1024, 16>::run(smem, args...);
-}
-
-template <int NT, int R>
-struct RegsSelect {
-    static dsa_status run(size_t smem, int32_t n_rows, const SelectArgs& a, cudaStream_t st)
-    {
-        dsa_status s = set_smem(select_regs_kernel<NT, R>, smem);
-        if (s != DSA_OK) return s;
-        DSA_LAUNCH(kProfSelect, st, launch_pdl(latency_bound(n_rows), select_regs_kernel<NT, R>, n_rows, NT, smem, st, a));
-        return launched();
-    }
-};
 
 template <int NT, int R>
 struct RegsHisaBlocks {

@@ -33,9 +33,15 @@
 // q . hi + q . mid + q . lo is the fp32 dot product up to accumulation order.
 // Every wait is bounded (1 s); a wait that runs out records an error in the
 // workspace status word and the CTA drains its copies and MMAs and exits.
+// A dense launch of one wave (decode) may do its own set-up (su.n_units > 0):
+// each CTA computes its unit from the layout, the first split of each query
+// tile writes the tile's rows for the select, CTA 0 clears the workspace
+// header, and the epilogue takes the eligible counts from the positions; the
+// call then needs no set-up kernel before it.
 #pragma once
 
 #include "ptx.cuh"
+#include "setup.cuh"
 
 namespace dsa {
 
@@ -122,7 +128,7 @@ enum : int { kTcTiles = 0, kTcGather = 1, kTcBlocks = 2 };
 template <int D, int H, int MODE>
 __global__ void __launch_bounds__(MODE == kTcGather ? kTcThreads : kTcThreadsTiles, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmKg, TcArgs a)
+                    const __grid_constant__ CUtensorMap tmKg, TcArgs a, const __grid_constant__ DenseSetupArgs su)
 {
     constexpr bool GATHER = MODE == kTcGather;
     constexpr bool EXT = MODE == kTcBlocks;
@@ -170,7 +176,21 @@ __global__ void __launch_bounds__(MODE == kTcGather ? kTcThreads : kTcThreadsTil
     if (warp == 1) tmem_alloc(tmem_slot, 512);
     grid_dep_wait();     // the unit table and rows come from earlier kernels
     // (no early launch of the next kernel: its CTAs waiting on freed SMs slowed decode down)
-    const TcUnit u = a.units[blockIdx.x];
+    const bool own_setup = !GATHER && !EXT && su.n_units > 0;
+    int seq_len = 0;     // own set-up: the unit's sequence length
+    TcUnit u;
+    if (own_setup) {
+        int seq;
+        u = dense_unit(su, blockIdx.x, seq, seq_len);
+        if (blockIdx.x == 0)   // the call's status word and select counters start at zero
+            for (int i = threadIdx.x; i < su.header_words; i += blockDim.x) su.header[i] = 0u;
+        if ((int)blockIdx.x % su.splits == 0 && (int)threadIdx.x < u.nrows) {   // the tile's rows, for the select
+            const int r = u.row0 + threadIdx.x;
+            su.rows[r] = RowDesc{r, seq, eligible_count(su.q_pos[r], seq_len), 0};
+        }
+    } else {
+        u = a.units[blockIdx.x];
+    }
     const bool active = u.kt1 > u.kt0 && u.nrows > 0;   // uniform over the CTA
     const int n_acc = u.nrows > NQA ? 2 : 1;
     uint8_t* sQ = smem;
@@ -356,10 +376,11 @@ __global__ void __launch_bounds__(MODE == kTcGather ? kTcThreads : kTcThreadsTil
         // the tile's head weights and eligible counts, shared by the 8 epilogue warps
         for (int i = threadIdx.x - 64; i < 2 * NQA * H; i += 256) {
             const int j = i / H;
-            sW[i] = j < u.nrows ? a.W[(int64_t)a.rows[u.row0 + j].qrow * H + (i % H)] : 0.f;
+            const int qrow = own_setup ? u.row0 + j : j < u.nrows ? a.rows[u.row0 + j].qrow : 0;
+            sW[i] = j < u.nrows ? a.W[(int64_t)qrow * H + (i % H)] : 0.f;
         }
         for (int j = threadIdx.x - 64; j < 2 * NQA; j += 256)
-            sNc[j] = j < u.nrows ? a.rows[u.row0 + j].ncols : 0;
+            sNc[j] = j >= u.nrows ? 0 : own_setup ? eligible_count(su.q_pos[u.row0 + j], seq_len) : a.rows[u.row0 + j].ncols;
         asm volatile("bar.sync 1, 256;" ::: "memory");   // named barrier of the epilogue warps only
         const int quarter = warp & 3;           // TMEM lanes this warp may read
         const int half = (warp - 2) >> 2;       // which 128 columns of an accumulator

@@ -417,7 +417,8 @@ __device__ __forceinline__ void sel_mark_all(int n, uint32_t* gtmap)
 // 4. Emits the marked columns in column order (all of gtmap, the first krem of eqmap), then pads
 // the row to k with -1 (and NaN scores).  Thread t owns a contiguous run of bitmap words; one
 // block-wide scan of its (> T, == T) counts gives both its output offset and its tie rank.  When
-// the row fits in stage (16-byte aligned, stage_words words: k, or 2k with scores) it is assembled
+// the row fits in stage (16-byte aligned, stage_words words: k, or 2k with scores, whose columns are
+// staged and read back all at once) it is assembled
 // there and written with coalesced 16-byte stores, else written directly.
 template <int NT>
 __device__ __forceinline__ void sel_emit(const SelectArgs& a, const RowDesc& rd, int r, const float* src, int n,
@@ -472,14 +473,13 @@ __device__ __forceinline__ void sel_emit(const SelectArgs& a, const RowDesc& rd,
             const int b = __ffs(bits) - 1;
             const int col = c0 + b;
             const int32_t key = per_word ? wbase + b : a.map.kind == kMapList ? lrow[col] : map_col(a.map, rd, col);
-            const float sc = osc ? key_score(score_key(__ldg(src + col))) : 0.f;
             if (!DSA_CHECK(out < (uint32_t)k && key >= 0, a.status, 202)) { ++out; continue; }   // output slot, key
-            if (staged) {
+            if (staged) {   // the column: its score is read in the write-out, every thread's loads together
                 stage[out] = key;
-                if (osc) stage[k + out] = __float_as_int(sc);
+                if (osc) stage[k + out] = col;
             } else {
                 oidx[out] = key;
-                if (osc) osc[out] = sc;
+                if (osc) osc[out] = key_score(score_key(__ldg(src + col)));
             }
             ++out;
         }
@@ -506,20 +506,19 @@ __device__ __forceinline__ void sel_emit(const SelectArgs& a, const RowDesc& rd,
             }
             *reinterpret_cast<int4*>(oidx + j) = v;
             if (osc) {
-                int4 f = *reinterpret_cast<const int4*>(stage + k + j);
-                if (j + 3 >= n_out) {
-                    f.x = j < n_out ? f.x : kNaN;
-                    f.y = j + 1 < n_out ? f.y : kNaN;
-                    f.z = j + 2 < n_out ? f.z : kNaN;
-                    f.w = j + 3 < n_out ? f.w : kNaN;
-                }
-                *reinterpret_cast<int4*>(osc + j) = f;
+                const int4 c = *reinterpret_cast<const int4*>(stage + k + j);
+                float4 f;
+                f.x = j < n_out ? key_score(score_key(__ldg(src + c.x))) : __int_as_float(kNaN);
+                f.y = j + 1 < n_out ? key_score(score_key(__ldg(src + c.y))) : __int_as_float(kNaN);
+                f.z = j + 2 < n_out ? key_score(score_key(__ldg(src + c.z))) : __int_as_float(kNaN);
+                f.w = j + 3 < n_out ? key_score(score_key(__ldg(src + c.w))) : __int_as_float(kNaN);
+                *reinterpret_cast<float4*>(osc + j) = f;
             }
         }
     } else {
         for (int j = tid; j < k; j += NT) {
             oidx[j] = j < n_out ? stage[j] : -1;
-            if (osc) osc[j] = __int_as_float(j < n_out ? stage[k + j] : kNaN);
+            if (osc) osc[j] = j < n_out ? key_score(score_key(__ldg(src + stage[k + j]))) : __int_as_float(kNaN);
         }
     }
 }

@@ -232,17 +232,16 @@ __global__ void __launch_bounds__(NT, 1) select_cluster_kernel(SelectArgs a, int
             const int b = __ffs(bits) - 1;
             const int col = cw + b;
             const int32_t key = per_word ? wbase + b : a.map.kind == kMapList ? lrow[col] : map_col(a.map, rd, col);
-            const float sc = osc ? key_score(score_key(__ldg(src + col))) : 0.f;
             if (!DSA_CHECK(out0 + out < (uint32_t)k && out < (uint32_t)cnt && key >= 0, a.status, 302)) {
                 ++out;
                 continue;
             }
-            if (staged) {
+            if (staged) {   // the column: its score is read in the write-out, every thread's loads together
                 stage[out] = key;
-                if (osc) stage[cnt + out] = __float_as_int(sc);
+                if (osc) stage[cnt + out] = col;
             } else {
                 oidx[out0 + out] = key;
-                if (osc) osc[out0 + out] = sc;
+                if (osc) osc[out0 + out] = key_score(score_key(__ldg(src + col)));
             }
             ++out;
         }
@@ -251,7 +250,7 @@ __global__ void __launch_bounds__(NT, 1) select_cluster_kernel(SelectArgs a, int
         __syncthreads();
         for (int j = tid; j < cnt; j += NT) {
             oidx[out0 + j] = stage[j];
-            if (osc) osc[out0 + j] = __int_as_float(stage[cnt + j]);
+            if (osc) osc[out0 + j] = key_score(score_key(__ldg(src + stage[cnt + j])));
         }
     }
     if (p == 0) {   // padding past the row's columns

@@ -42,6 +42,31 @@ struct DenseSetupArgs {
     int32_t tile_base[kSetupMaxSeqs + 1];   // first tile of each sequence (tiles cut per sequence)
 };
 
+// Work unit u of a dense launch (u < a.n_units), computed alone; seq and L receive its sequence and
+// that sequence's key count.
+__device__ __forceinline__ TcUnit dense_unit(const DenseSetupArgs& a, int u, int& seq, int& L)
+{
+    const int tau = u / a.splits, s = u % a.splits;
+    int lo = 0, hi = a.n_seqs - 1;   // the sequence whose tiles hold tile tau
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.tile_base[mid] <= tau) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo;
+    const int q0 = a.q_off[b], nq = a.q_off[b + 1] - q0;
+    const int ntile = a.tile_base[b + 1] - a.tile_base[b];
+    const int jj = ntile - 1 - (tau - a.tile_base[b]);   // longest causal tiles first
+    const int r0 = q0 + jj * a.TQ;
+    const int nr = min(a.TQ, nq - jj * a.TQ);
+    const int kb = a.k_off[b];
+    L = a.k_off[b + 1] - kb;
+    seq = b;
+    int maxnc = 0;
+    for (int r = r0; r < r0 + nr; ++r) maxnc = max(maxnc, eligible_count(a.q_pos[r], L));
+    const int nkt = (maxnc + 127) / 128;
+    return TcUnit{r0, nr, nkt * s / a.splits, nkt * (s + 1) / a.splits, r0, kb, {0, 0}};
+}
+
 __global__ void dense_setup_kernel(const __grid_constant__ DenseSetupArgs a)
 {
     grid_dep_launch();   // the scoring kernel may set up; it waits for this grid before reading units
@@ -53,23 +78,8 @@ __global__ void dense_setup_kernel(const __grid_constant__ DenseSetupArgs a)
         a.rows[gid] = RowDesc{gid, b, eligible_count(a.q_pos[gid], a.k_off[b + 1] - a.k_off[b]), 0};
     }
     if (gid < a.n_units) {
-        const int tau = gid / a.splits, s = gid % a.splits;
-        int lo = 0, hi = a.n_seqs - 1;   // the sequence whose tiles hold tile tau
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (a.tile_base[mid] <= tau) lo = mid; else hi = mid - 1;
-        }
-        const int b = lo;
-        const int q0 = a.q_off[b], nq = a.q_off[b + 1] - q0;
-        const int ntile = a.tile_base[b + 1] - a.tile_base[b];
-        const int jj = ntile - 1 - (tau - a.tile_base[b]);   // longest causal tiles first
-        const int r0 = q0 + jj * a.TQ;
-        const int nr = min(a.TQ, nq - jj * a.TQ);
-        const int L = a.k_off[b + 1] - a.k_off[b];
-        int maxnc = 0;
-        for (int r = r0; r < r0 + nr; ++r) maxnc = max(maxnc, eligible_count(a.q_pos[r], L));
-        const int nkt = (maxnc + 127) / 128;
-        a.units[gid] = TcUnit{r0, nr, nkt * s / a.splits, nkt * (s + 1) / a.splits, r0, a.k_off[b], {0, 0}};
+        int seq, L;
+        a.units[gid] = dense_unit(a, gid, seq, L);
     }
 }
 
