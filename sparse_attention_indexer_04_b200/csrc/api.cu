@@ -230,20 +230,21 @@ dsa_status launch_score(const RowDesc* rows, int32_t n_rows, int32_t max_cols, c
     return launched();
 }
 
-// Threads per row of the streaming select: 256 when rows fill the GPU several times over, 512
-// when there are few rows or k is large (each row's phases are latency-bound), 1024 for k of 8192
-// or more (the candidate buffer then takes most of the shared memory: one CTA per SM).  Measured on
-// the 32K prefill (32768 rows: 256 best), the 16 x 32K decode (32 rows: 512 best) and PIVOT's
-// top-8192 candidate selection at 128K (1024: 3.12 ms against 3.44 with 512).
-int select_threads(int32_t n_rows, int32_t k)
-{
-    return k >= 8192 ? 1024 : n_rows < 2 * 148 || k >= 4096 ? 512 : 256;
-}
-
 // Dynamic shared memory the select kernels may take: a CTA's 227 KB less their static shared
 // memory (SelScalars: the radix histogram and scalars, about 1.2 KB; 4 KB reserved).
 constexpr size_t kSelectDynMax = (size_t)227 * 1024 - 4096;
 static_assert(sizeof(SelScalars<512>) + 512 <= 4096, "select static shared memory");
+
+// Threads per row of the streaming select: 256 when rows fill the GPU several times over, 512
+// when there are few rows, k is large or the shared memory leaves at most two CTAs per SM (each
+// row's phases are latency-bound), 1024 for k of 8192 or more (the candidate buffer then takes
+// most of the shared memory: one CTA per SM).  Measured on the 32K prefill (32768 rows: 256 best),
+// the 16 x 32K decode (32 rows: 512 best) and PIVOT's top-8192 candidate selection at 128K (1024:
+// 3.12 ms against 3.44 with 512).
+int select_threads(int32_t n_rows, int32_t k, size_t smem)
+{
+    return k >= 8192 ? 1024 : n_rows < 2 * 148 || k >= 4096 || smem > kSelectDynMax / 3 ? 512 : 256;
+}
 
 // Candidate buffer entries of the select: 1.75 k, or what fits in shared memory next to the
 // bitmaps of max_cols columns (a smaller buffer only sends more rows down the full-row path).
@@ -349,7 +350,7 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
                                                sp.ctr, P));
         return launched();
     }
-    switch (select_threads(n_rows, k)) {
+    switch (select_threads(n_rows, k, smem)) {
     case 1024:
         if ((s = set_smem(select_stream_kernel<1024>, smem)) != DSA_OK) return s;
         DSA_LAUNCH(kProfSelect, st, launch_pdl(latency_bound(n_rows), select_stream_kernel<1024>, n_rows, 1024, smem, st, a));
@@ -799,6 +800,10 @@ size_t pivot_plan(char* base, const dsa_batch* b, const HostInfo& hi, int32_t k,
 // status area, which every call clears before its first launch.
 int32_t* reuse_fallback_count(void* ws) { return reinterpret_cast<int32_t*>(static_cast<char*>(ws) + 64); }
 
+// Reuse without a candidate list: the groups the gated top-C selection ranks (0, or all of them once
+// some query needs the per-query selection); the next word of the status area.
+int32_t* reuse_gate(void* ws) { return reinterpret_cast<int32_t*>(static_cast<char*>(ws) + 68); }
+
 struct HisaPlan {
     int32_t* block_base;
     RowDesc* block_rows;
@@ -949,6 +954,55 @@ dsa_status dense_topk_one_launch(const dsa_batch* b, const HostInfo& hi, const T
                  hi.max_k, p.S, ld, p.units, p.tile_base, status, st, o);
     if (s != DSA_OK) return s;
     return launch_select(p.rows, b->num_queries, hi.max_k, k, ColMap{}, p.S, ld, false, idx, k, scores, k, st, p.split);
+}
+
+// PIVOT Reuse when the caller wants no candidate list (pivot_group_index, mode 0, cand NULL).  The
+// scan's scores stay in the buffer; the group's top k + G - 1 are selected from the proxy row
+// directly (no top-C selection); the Reuse kernel serves every query whose prefix keeps k of them.
+// Only if some query is left over (ragged positions) does a gated top-C selection build the
+// candidate lists, after which those queries are ranked one by one as in the listed path.
+dsa_status reuse_direct(const dsa_batch* b, const HostInfo& hi, const void* K, int32_t k, int32_t G, int32_t C,
+                        int32_t ng, const TcSource& src, int32_t* idx, const PivotPlan& p, void* ws, cudaStream_t st)
+{
+    uint32_t* status = static_cast<uint32_t*>(ws);
+    const int64_t ld = score_ld(hi.max_k);
+    dsa_status s = tc_score(p.proxy_rows, ng, 0, src, b->num_heads, b->head_dim, K, b->num_keys, b->k_offsets,
+                            ColMap{}, hi.max_k, p.S, ld, p.units, p.tile_base, status, st);
+    if (s != DSA_OK) return s;
+    const int32_t kp = reuse_list_len(k, G, C);
+    if ((s = launch_select(p.proxy_rows, ng, hi.max_k, kp, identity_map(), p.S, ld, false, p.gsel, kp, p.gscore, kp,
+                           st)) != DSA_OK)
+        return s;
+    const unsigned gq = (b->num_queries + 255) / 256;
+    DSA_LAUNCH(kProfSetup, st, pivot_query_rows_kernel<<<gq, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos,
+                                                                           b->num_seqs, b->num_queries, G, p.group_base,
+                                                                           nullptr, C, nullptr, p.query_rows));
+    if ((s = launched()) != DSA_OK) return s;
+    DSA_LAUNCH(kProfSetup, st, pivot_cand_rows_kernel<<<(ng + 255) / 256, 256, 0, st>>>(p.groups, ng, C, p.cand_rows));
+    if ((s = launched()) != DSA_OK) return s;
+    ReuseArgs ra{};
+    ra.groups = p.groups; ra.query_rows = p.query_rows; ra.cand_rows = p.cand_rows;
+    ra.gsel = p.gsel; ra.gscore = p.gscore; ra.kp = kp; ra.k = k; ra.cand = nullptr; ra.C = C;
+    ra.n_groups = ng; ra.gate = reuse_gate(ws);
+    ra.idx = idx; ra.ld_idx = k; ra.fb_rows = p.fb_rows; ra.fb_count = reuse_fallback_count(ws);
+    ra.status = status;
+    const size_t smem = reuse_smem_bytes(kp);
+    if ((s = set_smem(pivot_reuse_kernel, smem)) != DSA_OK) return s;
+    DSA_LAUNCH(kProfSelect, st, pivot_reuse_kernel<<<ng, kReuseThreads, smem, st>>>(ra));
+    if ((s = launched()) != DSA_OK) return s;
+    // left-over queries: the candidate lists (every group, or none when the gate stayed shut), their rows, their top k
+    if ((s = launch_select(p.proxy_rows, ng, hi.max_k, C, identity_map(), p.S, ld, false, p.cand, C, p.cand_score, C,
+                           st, SelectSplit{}, reuse_gate(ws))) != DSA_OK)
+        return s;
+    DSA_LAUNCH(kProfSetup, st, reuse_fallback_rows_kernel<<<gq, 256, 0, st>>>(p.fb_rows, reuse_fallback_count(ws),
+                                                                              p.cand, C));
+    if ((s = launched()) != DSA_OK) return s;
+    ColMap m{};
+    m.kind = kMapList;
+    m.list = p.cand;
+    m.list_ld = C;
+    return launch_select(p.fb_rows, b->num_queries, C, k, m, p.cand_score, C, true, idx, k, nullptr, 0, st,
+                         SelectSplit{}, reuse_fallback_count(ws));
 }
 
 // PIVOT Refine's second stage: each query scores its eligible candidates (query_rows, list map m)
@@ -1395,6 +1449,10 @@ dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, c
     if (ng == 0) return DSA_OK;
     const int H = b->num_heads, D = b->head_dim;
     int32_t* cand = cand_out ? cand_out : p.cand;
+    const int64_t ld = score_ld(hi.max_k);
+    // Reuse with no candidate list wanted, the scan's scores held at once: the group's list comes
+    // from the proxy row itself (the top k + G - 1 of the top C are the top k + G - 1 of the row)
+    const bool direct = mode == 0 && !cand_out && chunk_rows(ng, ld) >= ng;
 
     DSA_LAUNCH(kProfSetup, st, pivot_groups_kernel<<<1, 256, 0, st>>>(b->q_offsets, b->k_offsets, b->q_pos, b->num_seqs, G, ng, p.group_base,
                                            p.groups, p.proxy_rows));
@@ -1404,6 +1462,7 @@ dsa_status pivot_group_index(const dsa_batch* b, const void* Q, const void* K, c
     // Shared scan: each proxy against its prefix, top-C kept with their proxy scores.
     const std::vector<int32_t> goff = group_offsets_host(b, G);
     const TcSource src{p.Qp, ng, p.Wp, p.group_base, goff.data(), b->num_seqs};
+    if (direct) return reuse_direct(b, hi, K, k, G, C, ng, src, idx, p, ws, st);
     s = tc_score_and_select(p.proxy_rows, ng, src, H, D, K, b->num_keys, b->k_offsets, ColMap{}, hi.max_k, p.S, p.units,
                             p.tile_base, static_cast<uint32_t*>(ws), C, cand, C, p.cand_score, st);
     if (s != DSA_OK) return s;

@@ -37,9 +37,12 @@ struct ReuseArgs {
     const float* gscore;         // [n_groups, kp]: their proxy scores
     int32_t kp;
     int32_t k;
-    const int32_t* cand;         // [n_groups, C] candidate key indices, ascending
+    const int32_t* cand;         // [n_groups, C] candidate key indices, ascending; NULL: the group's list was
+                                 // selected from the proxy row itself, so gsel holds key indices (a query's
+                                 // row then has ncols = its key limit) and no candidate list exists yet
     int32_t C;
-    int32_t pad_;
+    int32_t n_groups;
+    int32_t* gate;               // (cand NULL) set to n_groups when some query is left to the per-query selection
     int32_t* idx;                // [n_q, ld_idx]
     int64_t ld_idx;
     RowDesc* fb_rows;            // queries left to the per-query selection
@@ -162,14 +165,17 @@ __global__ void __launch_bounds__(kReuseThreads) pivot_reuse_kernel(ReuseArgs a)
                 s_m = m;
                 s_drop = drop;
                 s_serve = serve ? 1 : 0;
-                if (!serve) a.fb_rows[atomicAdd(a.fb_count, 1)] = rd;
+                if (!serve) {
+                    a.fb_rows[atomicAdd(a.fb_count, 1)] = rd;
+                    if (a.gate) *a.gate = a.n_groups;   // the candidate lists are needed after all
+                }
             }
         }
         __syncthreads();
         if (s_serve) {
             const int m = s_m, drop = s_drop;
             int32_t* o = a.idx + (int64_t)t * a.ld_idx;
-            const int32_t* cl = a.cand + (int64_t)g * a.C;
+            const int32_t* cl = a.cand ? a.cand + (int64_t)g * a.C : nullptr;
             for (int i = tid; i < m; i += NT) {
                 int lo = 0, hi = drop;   // dropped positions before i
                 while (lo < hi) {
@@ -177,13 +183,32 @@ __global__ void __launch_bounds__(kReuseThreads) pivot_reuse_kernel(ReuseArgs a)
                     if (drop_pos[mid] < i) lo = mid + 1; else hi = mid;
                 }
                 if (lo < drop && drop_pos[lo] == i) continue;
-                if (!DSA_CHECK(i - lo < k && col[i] >= 0 && col[i] < a.C, a.status, 402)) continue;
-                o[i - lo] = cl[col[i]];
+                if (!DSA_CHECK(i - lo < k && col[i] >= 0 && (!a.cand || col[i] < a.C), a.status, 402)) continue;
+                o[i - lo] = a.cand ? cl[col[i]] : col[i];
             }
             for (int i = m - drop + tid; i < k; i += NT) o[i] = -1;
         }
         __syncthreads();
     }
+}
+
+// Reuse without a requested candidate list: the queries left to the per-query selection were listed
+// with their key limit as ncols; once the candidate lists exist (a top-C selection gated on those
+// queries), ncols becomes the count of the group's candidates below that limit.
+__global__ void reuse_fallback_rows_kernel(RowDesc* fb_rows, const int32_t* fb_count, const int32_t* cand, int32_t C)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= *fb_count) return;
+    RowDesc r = fb_rows[i];
+    const int32_t* c = cand + (int64_t)r.list * C;
+    int lo = 0, hi = C;   // first position whose candidate is >= the limit or -1
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        const int32_t s = c[mid];
+        if (s >= 0 && s < r.ncols) lo = mid + 1; else hi = mid;
+    }
+    r.ncols = lo;
+    fb_rows[i] = r;
 }
 
 }  // namespace dsa

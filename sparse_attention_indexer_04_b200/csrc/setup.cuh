@@ -205,6 +205,10 @@ __global__ void pivot_query_rows_kernel(const int32_t* q_off, const int32_t* k_o
     const int b = find_seq(q_off, n_seqs, t);
     const int g = group_base[b] + (t - q_off[b]) / G;
     const int lim = eligible_count(q_pos[t], k_off[b + 1] - k_off[b]);   // keys s < lim
+    if (!cand) {   // no candidate list yet: the row's limit in key indices
+        rows[t] = RowDesc{t, b, lim, g};
+        return;
+    }
     const int32_t* c = cand + (int64_t)g * C;
     int lo = 0, hi = cand_len ? cand_len[g] : C;   // first position whose candidate is >= lim or -1
     while (lo < hi) {

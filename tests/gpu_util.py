@@ -32,6 +32,13 @@ class Dev:
         torch.cuda.synchronize()
         return idx.cpu().numpy(), cand.cpu().numpy()
 
+    def pivot_idx(self, k, G, C, mode):
+        """Indices only (no candidate list asked for: Reuse then selects the group lists from the proxy
+        rows directly)."""
+        idx = dsa.pivot_group_index(self.lay, self.Q, self.K, self.W, k, G, C, mode)
+        torch.cuda.synchronize()
+        return idx.cpu().numpy()
+
     def hisa(self, k, B, keep):
         pooled = dsa.hisa_pool_keys(self.lay, self.K, B)
         idx, kept = dsa.hisa_index(self.lay, self.Q, self.K, self.W, pooled, k, B, keep, want_kept=True)

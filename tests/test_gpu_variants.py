@@ -68,6 +68,23 @@ def test_pivot_random_positions_exact(mode):
     check_exact_sets(idx, (ref["reuse_idx"] if mode == 0 else ref["refine_idx"])[group_rows(b, G)], "idx")
 
 
+@pytest.mark.parametrize("case", ["tiny", "ragged_random", "long_groups"])
+def test_pivot_reuse_without_candidate_list_exact(case):
+    """Reuse with no candidate list asked for selects each group's list from the proxy row itself and
+    builds candidate lists only for queries the list does not serve (scattered positions); integer
+    inputs, exact against the oracle."""
+    if case == "tiny":
+        b, (G, C, k) = workloads.tiny_integer(seed=5, T=512, H=4, d=32, k=64), (16, 256, 64)
+    elif case == "ragged_random":
+        b, (G, C, k) = workloads.ragged(41, [40, 24, 9], [300, 150, 64], H=4, d=32, k=24, integer=True,
+                                        pos_mode="random"), (8, 64, 24)
+    else:
+        b, (G, C, k) = workloads.tiny_integer(seed=9, T=2048, H=4, d=32, k=128), (16, 512, 128)
+    idx = Dev(b).pivot_idx(k, G, C, 0)
+    ref = oracle.pivot(b, G, C, k)
+    check_exact_sets(idx, ref["reuse_idx"][group_rows(b, G)], "idx")
+
+
 def _random_candidates(b, G, C, seed, bad_group=None):
     """Per group: a sorted random subset of its sequence's keys (some past its queries' positions), -1
     padded; with bad_group, that group's list has a descending pair in the middle."""
@@ -202,6 +219,8 @@ def test_full_size_pivot_128k_sampled_groups():
     reuse = dev.pivot(k, G, C, 0)
     refine = dev.pivot(k, G, C, 1)
     assert np.array_equal(reuse[1], refine[1])            # both modes share the candidate stage
+    # Reuse with no candidate list asked for: the same indices, row for row
+    assert np.array_equal(dev.pivot_idx(k, G, C, 0), reuse[0])
     check_pivot_bf16(b, G, C, k, 0, groups=groups, gpu=reuse)
     check_pivot_bf16(b, G, C, k, 1, groups=groups, gpu=refine)
 
