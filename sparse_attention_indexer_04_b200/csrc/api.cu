@@ -338,10 +338,16 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
         // the rows are long: measured, 16 x 128K 31-33 -> 27-28 us, 16 x 32K unchanged, and HISA's
         // ~8.4K-column token rows 3 us slower (ten cluster barriers against a short scan)
         const int chunk_words = ((((max_cols + P - 1) / P + 127) & ~127) + 31) / 32;
-        const size_t csmem = cluster_smem_bytes(a.sample_bytes, a.buf_cap, chunk_words);
+        // every CTA ranks the whole sample, so the cluster takes a smaller one (cluster_sample_size)
+        // and a candidate buffer of 3k entries for the wider threshold, as far as shared memory allows
+        SelectArgs ca = a;
+        ca.sample_bytes = cluster_sample_size(std::max(max_cols, 1), k) * 4;
+        const int64_t fit = (int64_t(kSelectDynMax) - ca.sample_bytes - int64_t(chunk_words) * 8) / 16;
+        ca.buf_cap = (int32_t)std::max<int64_t>(a.buf_cap, std::min<int64_t>((3 * int64_t(k) + 255) & ~255, fit & ~255));
+        const size_t csmem = cluster_smem_bytes(ca.sample_bytes, ca.buf_cap, chunk_words);
         if (P <= kClusterMaxParts && max_cols >= 16384 && csmem <= kSelectDynMax) {
             if ((s = set_smem(select_cluster_kernel<512>, csmem)) != DSA_OK) return s;
-            DSA_LAUNCH(kProfSelect, st, launch_clustered(select_cluster_kernel<512>, n_rows * P, 512, csmem, P, st, a,
+            DSA_LAUNCH(kProfSelect, st, launch_clustered(select_cluster_kernel<512>, n_rows * P, 512, csmem, P, st, ca,
                                                          P, chunk_words));
             return launched();
         }

@@ -44,6 +44,14 @@ __host__ __device__ inline int select_sample_size(int n, int k)
     return m < kSampleMin ? kSampleMin : (m > kSampleMax ? kSampleMax : (int)m);
 }
 
+// Sample of the cluster select (decode rows of up to 256K columns): at most 4096, since every CTA
+// of the cluster ranks the whole sample; its candidate buffer is sized for the wider threshold.
+__host__ __device__ inline int cluster_sample_size(int n, int k)
+{
+    const int m = select_sample_size(n, k);
+    return n <= 262144 && m > 4096 ? 4096 : m;
+}
+
 // Candidate buffer entries for top-k: at least 4096 and 1.75 k.
 __host__ __device__ inline int select_buf_cap(int k)
 {
@@ -222,12 +230,12 @@ struct alignas(16) SelScalars {
 // margin).
 template <int NT>
 __device__ __forceinline__ uint32_t sel_threshold(const float* src, int n, int k, int buf_cap, uint32_t* sample,
-                                                  SelScalars<NT>& sh)
+                                                  SelScalars<NT>& sh, int m_given = 0)
 {
     if (n <= buf_cap) return 0u;
     static_assert(NT >= 256 && kSampleMax / NT <= 32, "one run start per lane");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int m = select_sample_size(n, k);   // a multiple of 2048
+    const int m = m_given > 0 ? m_given : select_sample_size(n, k);   // a multiple of 2048
     // m / 32 evenly spaced runs of 32 consecutive columns (a warp reads one run: one or two cache
     // lines instead of 32 scattered sectors); run r starts at floor(r n / R) rounded down to 32.
     // Sample entry e belongs to run e / 32, so a warp's i-th run is warp + i NT / 32; lane i

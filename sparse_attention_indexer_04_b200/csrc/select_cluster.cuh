@@ -25,6 +25,11 @@ namespace cg = cooperative_groups;
 
 constexpr int kClusterMaxParts = 8;
 
+// The two halves of a cluster barrier: every thread of every CTA arrives (release), and a later
+// wait (acquire) returns once all have arrived; the work between them overlaps the barrier.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
 // Scalars the row's CTAs exchange; the leader's copy is the one read.
 struct alignas(16) ClusterShared {
     uint32_t gt[kClusterMaxParts];   // each CTA's marked counts (> T, == T)
@@ -81,17 +86,20 @@ __global__ void __launch_bounds__(NT, 1) select_cluster_kernel(SelectArgs a, int
             cs.overflow = 0;
         }
     }
-    cl.sync();   // the leader's counters are zero before any CTA adds to them
+    // the leader's counters are zero (and every CTA of the cluster runs) before any CTA touches the
+    // leader's shared memory: arrive now, wait just before the first such access
+    cluster_arrive();
 
     // ---- 1. tau: every CTA ranks the whole sample itself, the same way, so every CTA holds the same
     // tau with no cluster exchange (measured: the sample split among the CTAs, its digits summed in the
     // leader across two cluster barriers each, was 2-3.5 us slower per row)
     uint32_t tau = 0;
-    if (n > k) tau = sel_threshold<NT>(src, n, k, cap, sample, sh);
+    if (n > k) tau = sel_threshold<NT>(src, n, k, cap, sample, sh, cluster_sample_size(n, k));
 
     // ---- 2. this chunk's candidates; 3. into the leader's buffer
     if (n > k) sel_append<NT>(src, c0, c1, tau, cand, cap, sh);
     __syncthreads();
+    cluster_wait();
     const uint32_t mine_c = sh.count;
     if (tid == 0) {
         uint32_t base = 0xffffffffu;
@@ -201,7 +209,7 @@ __global__ void __launch_bounds__(NT, 1) select_cluster_kernel(SelectArgs a, int
         ties_before += eq_q;
     }
     const uint32_t quota = min(E, (uint32_t)max(0, krem - (int)ties_before));
-    cl.sync();   // nothing reads the leader's shared memory after this
+    cluster_arrive();   // this CTA reads the leader's shared memory no more; the wait is at the end
 
     // ---- this chunk's columns, at out0 + (earlier threads' columns)
     int32_t* oidx = a.out_idx + (int64_t)r * a.ld_idx;
@@ -259,6 +267,7 @@ __global__ void __launch_bounds__(NT, 1) select_cluster_kernel(SelectArgs a, int
             if (osc) osc[j] = __int_as_float(0x7fc00000);
         }
     }
+    cluster_wait();   // the leader's shared memory outlives every read of it
 }
 
 }  // namespace dsa
