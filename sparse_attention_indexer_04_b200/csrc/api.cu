@@ -330,7 +330,19 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
     a.out_from_qrow = n_rows_dev ? 1 : 0;
     a.buf_cap = select_cap(k, max_cols);
     a.sample_bytes = (int32_t)select_sample_bytes(std::max(max_cols, 1), k);
-    const size_t smem = select_smem_bytes(std::max(max_cols, 1), a.buf_cap, k);
+    size_t smem = select_smem_bytes(std::max(max_cols, 1), a.buf_cap, k);
+    const int m_cap = capped_sample_size(std::max(max_cols, 1), k);
+    if (m_cap * 4 < a.sample_bytes && n_rows > 2 * 148) {
+        // many long rows (PIVOT's group lists): a sample of at most 4096 columns and a candidate buffer
+        // of 3k entries for the wider threshold, in the same shared memory (the ranking of the sample
+        // is the one-CTA select's largest fixed cost per row)
+        const size_t words = (size_t(std::max(max_cols, 1)) + 31) / 32;
+        const int64_t fit = (int64_t(kSelectDynMax) - int64_t(m_cap) * 4 - int64_t(words) * 8) / 8;
+        a.capped_sample = 1;
+        a.sample_bytes = m_cap * 4;
+        a.buf_cap = (int32_t)std::max<int64_t>(a.buf_cap, std::min<int64_t>((3 * int64_t(k) + 255) & ~255, fit & ~255));
+        smem = size_t(a.sample_bytes) + size_t(a.buf_cap) * 8 + words * 8;
+    }
     dsa_status s;
     const int P = select_parts(n_rows, max_cols);
     if (sp.buf && sp.ctr && n_rows <= sp.max_rows && P > 1 && !n_rows_dev) {
@@ -338,10 +350,10 @@ dsa_status launch_select(const RowDesc* rows, int32_t n_rows, int32_t max_cols, 
         // the rows are long: measured, 16 x 128K 31-33 -> 27-28 us, 16 x 32K unchanged, and HISA's
         // ~8.4K-column token rows 3 us slower (ten cluster barriers against a short scan)
         const int chunk_words = ((((max_cols + P - 1) / P + 127) & ~127) + 31) / 32;
-        // every CTA ranks the whole sample, so the cluster takes a smaller one (cluster_sample_size)
+        // every CTA ranks the whole sample, so the cluster takes a smaller one (capped_sample_size)
         // and a candidate buffer of 3k entries for the wider threshold, as far as shared memory allows
         SelectArgs ca = a;
-        ca.sample_bytes = cluster_sample_size(std::max(max_cols, 1), k) * 4;
+        ca.sample_bytes = capped_sample_size(std::max(max_cols, 1), k) * 4;
         const int64_t fit = (int64_t(kSelectDynMax) - ca.sample_bytes - int64_t(chunk_words) * 8) / 16;
         ca.buf_cap = (int32_t)std::max<int64_t>(a.buf_cap, std::min<int64_t>((3 * int64_t(k) + 255) & ~255, fit & ~255));
         const size_t csmem = cluster_smem_bytes(ca.sample_bytes, ca.buf_cap, chunk_words);

@@ -44,9 +44,10 @@ __host__ __device__ inline int select_sample_size(int n, int k)
     return m < kSampleMin ? kSampleMin : (m > kSampleMax ? kSampleMax : (int)m);
 }
 
-// Sample of the cluster select (decode rows of up to 256K columns): at most 4096, since every CTA
-// of the cluster ranks the whole sample; its candidate buffer is sized for the wider threshold.
-__host__ __device__ inline int cluster_sample_size(int n, int k)
+// A smaller sample for rows of up to 256K columns: at most 4096, the candidate buffer sized for the
+// wider threshold.  Every CTA of the cluster select ranks the whole sample; the one-CTA select takes
+// it for long rows (PIVOT's group lists over 128K proxy rows).
+__host__ __device__ inline int capped_sample_size(int n, int k)
 {
     const int m = select_sample_size(n, k);
     return n <= 262144 && m > 4096 ? 4096 : m;
@@ -75,7 +76,7 @@ struct SelectArgs {
     int64_t ld_score;
     const int32_t* n_rows_dev;   // nullable: rows [*n_rows_dev, n_rows) are skipped (a count a kernel wrote)
     int32_t out_from_qrow;       // 1: row r writes output row rows[r].qrow instead of r
-    int32_t pad_;
+    int32_t capped_sample;       // 1: the one-CTA select samples capped_sample_size columns (long rows)
     uint32_t* status;            // the workspace status word (checked builds record index errors there)
 };
 
@@ -557,7 +558,8 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_stream_kernel(SelectArgs
     for (int w = threadIdx.x; w < 2 * nwords; w += NT) gtmap[w] = 0;
     int krem = n;   // ties at T still to take (every column when n <= k)
     if (n > k) {
-        const uint32_t tau = sel_threshold<NT>(src, n, k, cap, sample, sh);
+        const uint32_t tau =
+            sel_threshold<NT>(src, n, k, cap, sample, sh, a.capped_sample ? capped_sample_size(n, k) : 0);
         if (threadIdx.x == 0) sh.count = 0;
         __syncthreads();
         sel_append<NT>(src, 0, n, tau, buf, cap, sh);

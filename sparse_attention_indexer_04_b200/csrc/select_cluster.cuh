@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(NT, 1) select_cluster_kernel(SelectArgs a, int
     // tau with no cluster exchange (measured: the sample split among the CTAs, its digits summed in the
     // leader across two cluster barriers each, was 2-3.5 us slower per row)
     uint32_t tau = 0;
-    if (n > k) tau = sel_threshold<NT>(src, n, k, cap, sample, sh, cluster_sample_size(n, k));
+    if (n > k) tau = sel_threshold<NT>(src, n, k, cap, sample, sh, capped_sample_size(n, k));
 
     // ---- 2. this chunk's candidates; 3. into the leader's buffer
     if (n > k) sel_append<NT>(src, c0, c1, tau, cand, cap, sh);
