@@ -128,6 +128,27 @@ __device__ __forceinline__ void tma_gather4_2d(void* dst, const CUtensorMap* map
 
 // L2 eviction policy "evict last" for the whole access (fraction 1.0): lines loaded with it are
 // evicted after normal ones.
+// Two fp32 values as one 64-bit register pair, and back; d = a * b + c on both halves at once (each
+// half one IEEE fp32 fused multiply-add, rounded to nearest even).
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_last()
 {
     uint64_t p;

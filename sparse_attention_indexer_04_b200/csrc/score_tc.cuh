@@ -410,14 +410,18 @@ __global__ void __launch_bounds__(MODE == kTcGather ? kTcThreads : kTcThreadsTil
                     const float* w = sW + j * H;
                     float s0 = 0.f, s1 = 0.f;
                     if constexpr (H % 4 == 0) {
+                        // even heads into s0, odd into s1, as one packed pair: each fma.rn.f32x2 does two
+                        // IEEE fp32 fmas, the same ones in the same order as two scalar chains
+                        uint64_t acc = 0;   // (s0, s1) = (+0, +0)
 #pragma unroll
                         for (int h = 0; h < H; h += 4) {
                             const float4 w4 = *reinterpret_cast<const float4*>(w + h);
-                            s0 = fmaf(w4.x, fmaxf(v[q * H + h], 0.f), s0);
-                            s1 = fmaf(w4.y, fmaxf(v[q * H + h + 1], 0.f), s1);
-                            s0 = fmaf(w4.z, fmaxf(v[q * H + h + 2], 0.f), s0);
-                            s1 = fmaf(w4.w, fmaxf(v[q * H + h + 3], 0.f), s1);
+                            acc = fma_f32x2(pack_f32x2(w4.x, w4.y),
+                                            pack_f32x2(fmaxf(v[q * H + h], 0.f), fmaxf(v[q * H + h + 1], 0.f)), acc);
+                            acc = fma_f32x2(pack_f32x2(w4.z, w4.w),
+                                            pack_f32x2(fmaxf(v[q * H + h + 2], 0.f), fmaxf(v[q * H + h + 3], 0.f)), acc);
                         }
+                        unpack_f32x2(acc, s0, s1);
                     } else {
 #pragma unroll
                         for (int h = 0; h < H; ++h) s0 = fmaf(w[h], fmaxf(v[q * H + h], 0.f), s0);
