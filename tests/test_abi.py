@@ -65,6 +65,16 @@ def test_workspace_sizes_are_positive_and_grow():
     assert dsa.hisa_num_blocks(host_layout([1, 1], [300, 128]), 128) == 3 + 1
 
 
+def test_hisa_workspace_holds_the_bf16_planes_of_the_pooled_keys():
+    """When HISA's stages each run in one launch (at most 480 sequences, rows of at most 16,384 blocks
+    and kept tokens) the workspace carries the pooled keys as three bf16 planes: 6 bytes per element."""
+    L, B = 262144, 128
+    lay = host_layout([2] * 4, [L] * 4, H=64, d=128, pos=torch.full((8,), L - 1, dtype=torch.int32))
+    blocks = dsa.hisa_num_blocks(lay, B)
+    assert blocks == 4 * L // B
+    assert dsa.hisa_index_workspace(lay, 2048, B, 64) >= 3 * blocks * 128 * 2
+
+
 @pytest.mark.parametrize("H,d,ok", [(4, 32, True), (64, 128, True), (3, 32, False), (4, 48, False),
                                     (128, 64, False)])
 def test_unsupported_shapes_rejected(H, d, ok):
